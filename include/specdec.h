@@ -1,0 +1,174 @@
+/*
+ * specdec.h -- C-ABI of libspecdec.so: the batched speculative-sampling verify
+ * step on an NVIDIA B200 (sm_100a).
+ *
+ * The operation (Leviathan et al., as restated on the speculative decoding blog
+ * page "Speculative Decoding ... Llama 70B x2.4", section "The mathematical
+ * definition from Leviathan et al. (Google DeepMind, 2023)"):
+ *
+ *   For each sequence b, with p_i = softmax(target_logits[b,i,:] / T_b) and
+ *   q_i = softmax(draft_logits[b,i,:] / T_b):
+ *     for i = 0..K-1: accept draft token x_i = draft_tokens[b,i] iff
+ *                     u_accept[b,i] * q_i(x_i) < p_i(x_i)
+ *                     (i.e. u < alpha(x) = min(1, p/q)); stop at the first
+ *                     rejection, at position n;
+ *     if n < K : draw y from the corrected distribution
+ *                p'(v) = max(0, p_n(v) - q_n(v)) / Z   ("resample");
+ *     if n == K: draw y from p_K, the target's extra row ("bonus" token, as
+ *                in the SMC-SD page "Faster LLM Inference via Sequential
+ *                Monte Carlo", section 2, scoring step);
+ *     the draw is the inverse CDF with the supplied uniform:
+ *                y = min{ j : sum_{v<=j} r(v) > u_resample[b] * sum_v r(v) },
+ *                sums in ascending token order.
+ *   Outputs: out_tokens[b,0..n-1] = x_0..x_{n-1}, out_tokens[b,n] = y,
+ *            out_tokens[b,n+1..K] = -1, out_num_accepted[b] = n.
+ *   Temperature applies to both models (the blog's vLLM example sets
+ *   temperature=0.7; its trade-off 4 discusses T=0.3..1.0).
+ *
+ * Layouts (all row-major, the vocabulary dimension contiguous):
+ *   target_logits    [B, K+1, V]  bf16 or fp32 (see specdec_dtype)
+ *   draft_logits     [B, K,   V]  same dtype as the target
+ *   draft_tokens     [B, K]       int32
+ *   u_accept         [B, K]       fp32 in [0, 1)
+ *   u_resample       [B]          fp32 in [0, 1)
+ *   temperature      [B]          fp32, finite and > 0 (one per sequence)
+ *   out_tokens       [B, K+1]     int32
+ *   out_num_accepted [B]          int32
+ *
+ * Ownership: every pointer is owned by the caller.  Unless a function says
+ * otherwise, pointers are DEVICE memory of the current CUDA device and the call
+ * is asynchronous on `stream` (a cudaStream_t; NULL is the legacy default
+ * stream): nothing is synchronised, results are valid once the stream reaches
+ * the end of the call.  The logit pointers must be aligned to their element
+ * size; 16-byte alignment of every row (V * element size a multiple of 16)
+ * gives the fast vector path, other layouts take a slower scalar path.
+ *
+ * Errors:
+ *   SPECDEC_EINVAL  an argument is invalid (checked on the host before any
+ *                   launch; nothing is written): a null pointer with B > 0,
+ *                   B < 0, K outside [1, 32], V < 1, sizes that overflow,
+ *                   misaligned logits, an unknown dtype.  B == 0 is a no-op.
+ *   SPECDEC_ECUDA   a CUDA runtime call failed (launch, allocation, copy).
+ *   SPECDEC_ESTATE  the library-owned workspace would have to grow while
+ *                   `stream` is being captured into a CUDA graph (call once
+ *                   with the same or larger sizes before capturing).
+ *   Per-sequence input errors are found on the device and never fault:
+ *   a draft token outside [0, V), a temperature that is not finite and > 0,
+ *   or a logit row holding NaN or +Inf or only -Inf make that sequence's
+ *   out_num_accepted -1 and all its out_tokens -1, and set a bit in a
+ *   per-device error word (see specdec_device_errors).
+ * Determinism: results are bit-identical for identical inputs and sizes.
+ */
+#ifndef SPECDEC_H
+#define SPECDEC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum specdec_status {
+  SPECDEC_OK = 0,
+  SPECDEC_EINVAL = 1,
+  SPECDEC_ECUDA = 2,
+  SPECDEC_EDEVICE = 3,
+  SPECDEC_ESTATE = 4
+} specdec_status;
+
+typedef enum specdec_dtype { SPECDEC_F32 = 0, SPECDEC_BF16 = 1 } specdec_dtype;
+
+/* bits of the per-device error word */
+#define SPECDEC_ERR_TOKEN 1u       /* a draft token outside [0, V)            */
+#define SPECDEC_ERR_TEMPERATURE 2u /* a temperature not finite and > 0        */
+#define SPECDEC_ERR_LOGITS 4u      /* a row with NaN / +Inf / only -Inf       */
+
+/* Optional diagnostics (device pointers, each nullable).  Row order per
+ * sequence: target rows 0..K, then draft rows 0..K-1.
+ *   row_max [B, 2K+1] float : max_v z_v
+ *   row_sum [B, 2K+1] double: sum_v exp((z_v - max) / T)
+ *   p_x, q_x [B, K]  double: p_i(x_i), q_i(x_i) for positions i <= n only
+ *                            (other entries are left untouched)
+ *   Z [B]            double: mass of the distribution drawn from,
+ *                            sum_v max(0, p_n - q_n) or sum_v p_K (~1)      */
+typedef struct specdec_debug {
+  float *row_max;
+  double *row_sum;
+  double *p_x;
+  double *q_x;
+  double *Z;
+} specdec_debug;
+
+/* The verify step (see the top of this file).  Uses a workspace owned by the
+ * library (one per device, grown on demand with cudaMalloc, which
+ * synchronises the device the first time a size is seen). */
+specdec_status specdec_verify(const void *target_logits, const void *draft_logits,
+                              const int32_t *draft_tokens, const float *u_accept,
+                              const float *u_resample, const float *temperature, int B, int K,
+                              int V, specdec_dtype dtype, int32_t *out_tokens,
+                              int32_t *out_num_accepted, void *stream);
+
+/* Same as specdec_verify with the dtype fixed. */
+specdec_status specdec_verify_bf16(const void *target_logits, const void *draft_logits,
+                                   const int32_t *draft_tokens, const float *u_accept,
+                                   const float *u_resample, const float *temperature, int B,
+                                   int K, int V, int32_t *out_tokens, int32_t *out_num_accepted,
+                                   void *stream);
+specdec_status specdec_verify_f32(const void *target_logits, const void *draft_logits,
+                                  const int32_t *draft_tokens, const float *u_accept,
+                                  const float *u_resample, const float *temperature, int B,
+                                  int K, int V, int32_t *out_tokens, int32_t *out_num_accepted,
+                                  void *stream);
+
+/* Bytes of device workspace specdec_verify_ex needs for these sizes
+ * (0 for invalid sizes). */
+size_t specdec_workspace_bytes(int B, int K, int V, specdec_dtype dtype);
+
+/* specdec_verify with a caller-owned workspace (device memory of at least
+ * specdec_workspace_bytes bytes, 256-byte aligned; its contents need no
+ * initialisation) and optional diagnostics (dbg may be NULL).  Allocates
+ * nothing.  Calls that share a workspace must not overlap on the device. */
+specdec_status specdec_verify_ex(const void *target_logits, const void *draft_logits,
+                                 const int32_t *draft_tokens, const float *u_accept,
+                                 const float *u_resample, const float *temperature, int B,
+                                 int K, int V, specdec_dtype dtype, void *workspace,
+                                 size_t workspace_bytes, const specdec_debug *dbg,
+                                 int32_t *out_tokens, int32_t *out_num_accepted, void *stream);
+
+/* End-to-end variant: every pointer is HOST memory (pinned memory makes the
+ * copies asynchronous).  Copies the inputs to library-owned device buffers,
+ * runs the verify step on `stream`, copies the outputs back and synchronises
+ * `stream` before returning. */
+specdec_status specdec_verify_host(const void *target_logits, const void *draft_logits,
+                                   const int32_t *draft_tokens, const float *u_accept,
+                                   const float *u_resample, const float *temperature, int B,
+                                   int K, int V, specdec_dtype dtype, int32_t *out_tokens,
+                                   int32_t *out_num_accepted, void *stream);
+
+/* Synchronise `stream`, then read and clear the current device's error word
+ * (SPECDEC_ERR_* bits) into *flags.  Returns SPECDEC_EDEVICE when a bit was set. */
+specdec_status specdec_device_errors(void *stream, uint32_t *flags);
+
+/* Free the library-owned workspaces and staging buffers of every device. */
+void specdec_release(void);
+
+const char *specdec_status_string(specdec_status s);
+
+/* Kernel accounting, for benchmarks.  The library has specdec_kernel_count()
+ * kernels; specdec_kernel_name(i) names kernel i.  specdec_launch_count(i)
+ * counts its launches since the library was loaded.  Between
+ * specdec_profile_begin(max) and specdec_profile_end, up to `max` launches per
+ * kernel are bracketed with CUDA events on their stream; profile_end
+ * synchronises those events and writes, per kernel, the summed device time in
+ * milliseconds and the number of timed launches. */
+int specdec_kernel_count(void);
+const char *specdec_kernel_name(int i);
+uint64_t specdec_launch_count(int i);
+specdec_status specdec_profile_begin(int max_launches_per_kernel);
+specdec_status specdec_profile_end(double *ms_per_kernel, int *launches_per_kernel, int n);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SPECDEC_H */

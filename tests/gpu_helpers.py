@@ -1,0 +1,137 @@
+"""Helpers shared by the GPU tests: move seeded inputs to the device, run the
+CUDA path through the C-ABI, run the oracle, and compare them."""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+import speculative_sampling_b200 as sd
+
+# Tolerance for probabilities (row normalisers, p(x), q(x), Z): 1e-5 relative.
+# The kernels widen logits exactly, carry log2(e)/T as two fp32 parts, evaluate
+# 2^x with ex2.approx (about 2 ulp, i.e. ~2.4e-7 relative per element), sum
+# each thread's elements in fp32 and every combine in fp64, so the expected
+# error of a normaliser is a few 1e-7 relative; 1e-5 leaves a wide margin while
+# still catching any dropped term or wrong scale.
+RTOL = 1e-5
+# Decisions whose oracle margin is below this band may legitimately differ.
+BAND = 1e-6
+
+
+def require_cuda():
+    import torch
+    if not torch.cuda.is_available():
+        raise RuntimeError("this test needs a CUDA device (B200)")
+    return torch
+
+
+def to_device(x):
+    torch = require_cuda()
+    dev = torch.device("cuda", 0)
+    if x.dtype == "bf16":
+        tg = torch.from_numpy(x.target.view(np.int16)).to(dev).view(torch.bfloat16)
+        dr = torch.from_numpy(x.draft.view(np.int16)).to(dev).view(torch.bfloat16)
+    else:
+        tg = torch.from_numpy(x.target).to(dev)
+        dr = torch.from_numpy(x.draft).to(dev)
+    return dict(
+        target=tg, draft=dr,
+        tokens=torch.from_numpy(np.ascontiguousarray(x.tokens)).to(dev),
+        u_accept=torch.from_numpy(x.u_accept).to(dev),
+        u_resample=torch.from_numpy(x.u_resample).to(dev),
+        temperature=torch.from_numpy(x.temperature).to(dev))
+
+
+def gpu_verify(x, debug=True, dev_inputs=None, garbage_workspace=False):
+    """CUDA path through specdec_verify_ex (with diagnostics) or specdec_verify."""
+    torch = require_cuda()
+    d = dev_inputs if dev_inputs is not None else to_device(x)
+    B, K = x.B, x.K
+    R = 2 * K + 1
+    dev = d["target"].device
+    out = {}
+    if debug:
+        dbg = dict(row_max=torch.full((B, R), float("nan"), dtype=torch.float32, device=dev),
+                   row_sum=torch.full((B, R), float("nan"), dtype=torch.float64, device=dev),
+                   p_x=torch.full((B, K), float("nan"), dtype=torch.float64, device=dev),
+                   q_x=torch.full((B, K), float("nan"), dtype=torch.float64, device=dev),
+                   Z=torch.full((B,), float("nan"), dtype=torch.float64, device=dev))
+        ws = None
+        if garbage_workspace:
+            dt = sd.SPECDEC_BF16 if x.dtype == "bf16" else sd.SPECDEC_F32
+            n = sd.specdec_workspace_bytes(B, K, x.V, dt)
+            ws = torch.randint(0, 255, (n,), dtype=torch.uint8, device=dev)
+        ot, on = sd.verify(d["target"], d["draft"], d["tokens"], d["u_accept"], d["u_resample"],
+                           d["temperature"], debug=dbg, workspace=ws)
+        torch.cuda.synchronize()
+        for k, v in dbg.items():
+            out[k] = v.cpu().numpy()
+    else:
+        ot, on = sd.verify(d["target"], d["draft"], d["tokens"], d["u_accept"], d["u_resample"],
+                           d["temperature"])
+        torch.cuda.synchronize()
+    out["out_tokens"] = ot.cpu().numpy()
+    out["num_accepted"] = on.cpu().numpy()
+    return out
+
+
+def oracle_verify(x, seqs=None, nthreads=8):
+    if seqs is None:
+        return oracle.verify(x.target, x.draft, x.tokens, x.u_accept, x.u_resample,
+                             x.temperature, dtype=x.dtype, nthreads=nthreads)
+    s = np.asarray(seqs)
+    return oracle.verify(x.target[s], x.draft[s], x.tokens[s], x.u_accept[s], x.u_resample[s],
+                         x.temperature[s], dtype=x.dtype, nthreads=nthreads)
+
+
+def rel(a, b):
+    """Relative difference; probabilities below 1e-200 count as equal to 0."""
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    return np.abs(a - b) / np.maximum(np.abs(b), 1e-200)
+
+
+def compare(g: dict, o: dict, seqs=None, rtol=RTOL, band=BAND, stats=True) -> dict:
+    """Element-by-element comparison of the CUDA path (g) with the oracle (o).
+
+    Integer outputs: bit-exact on every sequence whose oracle decisions are not
+    within ``band`` of a threshold; such boundary draws are counted.  Invalid
+    sequences (n = -1) must agree exactly.  Probabilities: within ``rtol``."""
+    if seqs is not None:
+        g = {k: v[np.asarray(seqs)] for k, v in g.items()}
+    on, gn = o["num_accepted"], g["num_accepted"]
+    assert np.array_equal(on < 0, gn < 0), "invalid-sequence verdicts differ"
+    assert np.all(g["out_tokens"][gn < 0] == -1)
+    valid = on >= 0
+    bnd = oracle.boundary_mask(o, band) & valid
+    exact = valid & ~bnd
+    mism = np.nonzero(exact & (np.any(g["out_tokens"] != o["out_tokens"], axis=1) | (gn != on)))[0]
+    assert mism.size == 0, (f"{mism.size} non-boundary sequences differ, e.g. seq {mism[:5]}: "
+                            f"gpu n={gn[mism[:5]]} oracle n={on[mism[:5]]} "
+                            f"gpu={g['out_tokens'][mism[:2]]} oracle={o['out_tokens'][mism[:2]]}")
+    K = o["out_tokens"].shape[1] - 1
+    # draws per valid sequence: min(n+1, K) acceptance tests + one token draw
+    draws = int(np.sum(np.minimum(on[valid] + 1, K) + 1))
+    differ = valid & (np.any(g["out_tokens"] != o["out_tokens"], axis=1) | (gn != on))
+    res = {"sequences": int(on.size), "valid": int(valid.sum()), "boundary": int(bnd.sum()),
+           "draws": draws, "mismatched": int(differ.sum())}
+    # Disagreements are allowed only on boundary draws, and must stay under
+    # 0.01% of all draws (with fewer than 10^4 draws: none at all).
+    assert res["mismatched"] <= int(1e-4 * draws), res
+    if not stats or "row_sum" not in g:
+        return res
+    v = valid
+    assert np.array_equal(g["row_max"][v].astype(np.float64), o["row_max"][v]), "row max"
+    e_s = rel(g["row_sum"][v], o["row_sum"][v])
+    assert e_s.max(initial=0) <= rtol, ("row sum", e_s.max())
+    same = exact | (v & (gn == on))
+    reach = (np.arange(K)[None, :] <= on[:, None]) & same[:, None]
+    e_p = rel(g["p_x"][reach], o["p_x"][reach])
+    e_q = rel(g["q_x"][reach], o["q_x"][reach])
+    assert e_p.max(initial=0) <= rtol, ("p(x)", e_p.max())
+    assert e_q.max(initial=0) <= rtol, ("q(x)", e_q.max())
+    e_z = rel(g["Z"][same], o["Z"][same])
+    assert e_z.max(initial=0) <= rtol, ("Z", e_z.max())
+    res.update(max_rel_row_sum=float(e_s.max(initial=0)), max_rel_px=float(e_p.max(initial=0)),
+               max_rel_qx=float(e_q.max(initial=0)), max_rel_Z=float(e_z.max(initial=0)))
+    return res
