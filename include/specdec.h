@@ -74,7 +74,8 @@ typedef enum specdec_status {
   SPECDEC_EINVAL = 1,
   SPECDEC_ECUDA = 2,
   SPECDEC_EDEVICE = 3,
-  SPECDEC_ESTATE = 4
+  SPECDEC_ESTATE = 4,
+  SPECDEC_ESIZE = 5
 } specdec_status;
 
 typedef enum specdec_dtype { SPECDEC_F32 = 0, SPECDEC_BF16 = 1 } specdec_dtype;
@@ -149,6 +150,36 @@ specdec_status specdec_verify_host(const void *target_logits, const void *draft_
 /* Synchronise `stream`, then read and clear the current device's error word
  * (SPECDEC_ERR_* bits) into *flags.  Returns SPECDEC_EDEVICE when a bit was set. */
 specdec_status specdec_device_errors(void *stream, uint32_t *flags);
+
+/* Allocation-free verify (no counterpart on the pages: an interface addition).
+ *
+ * For callers that cannot allocate device memory -- for example a serving
+ * engine that has handed nearly all of HBM to its own pools (KV cache) and
+ * forbids allocations behind its back, or a latency-critical loop that cannot
+ * afford cudaMalloc's device-wide synchronisation.  Same arguments and results
+ * as specdec_verify, but the workspace is a fixed device array inside the
+ * library (SPECDEC_STATIC_SCRATCH_BYTES, 4 MiB, held by every device that
+ * loads the library until the process exits); the call itself never calls
+ * cudaMalloc, cudaFree or any allocating routine.  The caller still provides
+ * every input and output buffer.
+ *   - Returns SPECDEC_ESIZE, launching nothing, when these sizes need more
+ *     workspace than the array holds (compare specdec_workspace_bytes with
+ *     SPECDEC_STATIC_SCRATCH_BYTES; B=64,K=5,V=128256 needs about 0.2 MiB,
+ *     B=256,K=8,V=151936 about 2.8 MiB).
+ *   - The first call on a device looks up the array's device address (once
+ *     per device, with that device current); make that first call before any
+ *     stream capture on that device.
+ *   - All calls share the one array, which keeps the last call's contents:
+ *     calls whose executions overlap on the GPU (on different streams, or
+ *     from different host threads) race on it and must be serialised by the
+ *     caller.  The kernels rewrite everything they read, so no clearing is
+ *     needed between calls. */
+#define SPECDEC_STATIC_SCRATCH_BYTES (4u << 20)
+specdec_status specdec_verify_static(const void *target_logits, const void *draft_logits,
+                                     const int32_t *draft_tokens, const float *u_accept,
+                                     const float *u_resample, const float *temperature, int B,
+                                     int K, int V, specdec_dtype dtype, int32_t *out_tokens,
+                                     int32_t *out_num_accepted, void *stream);
 
 /* Free the library-owned workspaces and staging buffers of every device. */
 void specdec_release(void);

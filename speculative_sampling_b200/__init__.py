@@ -17,7 +17,8 @@ from typing import Optional
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libspecdec.so")
 
-SPECDEC_OK, SPECDEC_EINVAL, SPECDEC_ECUDA, SPECDEC_EDEVICE, SPECDEC_ESTATE = range(5)
+SPECDEC_OK, SPECDEC_EINVAL, SPECDEC_ECUDA, SPECDEC_EDEVICE, SPECDEC_ESTATE, SPECDEC_ESIZE = range(6)
+SPECDEC_STATIC_SCRATCH_BYTES = 4 << 20
 SPECDEC_F32, SPECDEC_BF16 = 0, 1
 SPECDEC_ERR_TOKEN, SPECDEC_ERR_TEMPERATURE, SPECDEC_ERR_LOGITS = 1, 2, 4
 
@@ -31,6 +32,7 @@ _SIGS = {
     "specdec_verify_ex": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, ctypes.c_size_t, _P,
                                _P, _P, _P]),
     "specdec_verify_host": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P]),
+    "specdec_verify_static": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P]),
     "specdec_device_errors": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
     "specdec_release": (None, []),
     "specdec_status_string": (ctypes.c_char_p, [_I]),
@@ -117,6 +119,15 @@ def specdec_verify_host(target, draft, tokens, u_accept, u_resample, temperature
                         dtype, out_tokens, out_num_accepted, stream) -> int:
     return lib().specdec_verify_host(target, draft, tokens, u_accept, u_resample, temperature,
                                      B, K, V, dtype, out_tokens, out_num_accepted, stream)
+
+
+def specdec_verify_static(target, draft, tokens, u_accept, u_resample, temperature, B, K, V,
+                          dtype, out_tokens, out_num_accepted, stream) -> int:
+    """specdec_verify with the library's fixed scratch instead of an allocated
+    workspace, for callers that may not allocate device memory (see the header
+    for the size limit and the no-overlap rule)."""
+    return lib().specdec_verify_static(target, draft, tokens, u_accept, u_resample, temperature,
+                                       B, K, V, dtype, out_tokens, out_num_accepted, stream)
 
 
 def specdec_device_errors(stream=None) -> tuple:

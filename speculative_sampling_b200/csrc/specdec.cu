@@ -896,6 +896,40 @@ specdec_status ensure_buf(std::unordered_map<int, DeviceBuf> &map, size_t bytes,
 }  // namespace
 
 // ---------------------------------------------------------------------------
+// Fixed scratch for specdec_verify_static.  Some callers cannot allocate device
+// memory at all: a serving engine that has reserved nearly all of HBM for its
+// own pools (KV cache) and forbids allocations behind its back, or a caller
+// that cannot afford cudaMalloc's device-wide synchronisation on its path.
+// For them the workspace lives in this module-level device array instead: it
+// is created when the module is loaded on a device and stays until the process
+// exits, on every device that loads the library.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_static_scratch[SPECDEC_STATIC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_static_mu;
+std::unordered_map<int, void *> g_static_addr;  // device -> address of g_static_scratch
+
+// Device address of the fixed scratch on the current device.  In host code the
+// array's name only stands for the symbol; its device address is looked up
+// once per device (with that device current) and cached.
+specdec_status static_scratch_address(void **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SPECDEC_ECUDA;
+  std::lock_guard<std::mutex> lk(g_static_mu);
+  auto it = g_static_addr.find(dev);
+  if (it == g_static_addr.end()) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr)
+      return SPECDEC_ECUDA;
+    it = g_static_addr.emplace(dev, p).first;
+  }
+  *out = it->second;
+  return SPECDEC_OK;
+}
+}  // namespace
+
+// ---------------------------------------------------------------------------
 // C-ABI
 // ---------------------------------------------------------------------------
 extern "C" {
@@ -1008,6 +1042,28 @@ specdec_status specdec_device_errors(void *stream, uint32_t *flags) {
   return v ? SPECDEC_EDEVICE : SPECDEC_OK;
 }
 
+specdec_status specdec_verify_static(const void *target_logits, const void *draft_logits,
+                                     const int32_t *draft_tokens, const float *u_accept,
+                                     const float *u_resample, const float *temperature, int B,
+                                     int K, int V, specdec_dtype dtype, int32_t *out_tokens,
+                                     int32_t *out_num_accepted, void *stream) {
+  specdec_status s = check_args(target_logits, draft_logits, draft_tokens, u_accept, u_resample,
+                                temperature, B, K, V, dtype, out_tokens, out_num_accepted);
+  if (s != SPECDEC_OK || B == 0) return s;
+  const size_t need = specdec_workspace_bytes(B, K, V, dtype);
+  if (need == 0) return SPECDEC_EINVAL;
+  if (need > (size_t)SPECDEC_STATIC_SCRATCH_BYTES) return SPECDEC_ESIZE;
+  void *scratch = nullptr;
+  s = static_scratch_address(&scratch);
+  if (s != SPECDEC_OK) return s;
+  // Nothing in the scratch has to start at zero: every record the kernels read
+  // (V-split partials, per-sequence selection, chunk sums, the arrival counters
+  // that k_accept resets) is written earlier in the same call.
+  return run(target_logits, draft_logits, draft_tokens, u_accept, u_resample, temperature, B, K,
+             V, dtype, scratch, (size_t)SPECDEC_STATIC_SCRATCH_BYTES, nullptr, out_tokens,
+             out_num_accepted, static_cast<cudaStream_t>(stream));
+}
+
 void specdec_release(void) {
   std::lock_guard<std::mutex> lk(g_mu);
   int cur = 0;
@@ -1032,6 +1088,7 @@ const char *specdec_status_string(specdec_status s) {
     case SPECDEC_ECUDA: return "CUDA runtime error";
     case SPECDEC_EDEVICE: return "invalid inputs flagged on the device";
     case SPECDEC_ESTATE: return "workspace would grow during stream capture";
+    case SPECDEC_ESIZE: return "sizes need more than the fixed scratch of specdec_verify_static";
   }
   return "unknown status";
 }
