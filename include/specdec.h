@@ -84,6 +84,8 @@ typedef enum specdec_dtype { SPECDEC_F32 = 0, SPECDEC_BF16 = 1 } specdec_dtype;
 #define SPECDEC_ERR_TOKEN 1u       /* a draft token outside [0, V)            */
 #define SPECDEC_ERR_TEMPERATURE 2u /* a temperature not finite and > 0        */
 #define SPECDEC_ERR_LOGITS 4u      /* a row with NaN / +Inf / only -Inf       */
+#define SPECDEC_ERR_TIMEOUT 8u     /* a bounded on-chip wait ran out: the
+                                      call's outputs are all -1              */
 
 /* Optional diagnostics (device pointers, each nullable).  Row order per
  * sequence: target rows 0..K, then draft rows 0..K-1.
@@ -164,8 +166,8 @@ specdec_status specdec_device_errors(void *stream, uint32_t *flags);
  * every input and output buffer.
  *   - Returns SPECDEC_ESIZE, launching nothing, when these sizes need more
  *     workspace than the array holds (compare specdec_workspace_bytes with
- *     SPECDEC_STATIC_SCRATCH_BYTES; B=64,K=5,V=128256 needs about 0.2 MiB,
- *     B=256,K=8,V=151936 about 2.8 MiB).
+ *     SPECDEC_STATIC_SCRATCH_BYTES; B=64,K=5,V=128256 needs about 0.05 MiB,
+ *     B=256,K=8,V=151936 about 0.4 MiB, B=2048,K=8,V=151936 about 3.4 MiB).
  *   - The first call on a device looks up the array's device address (once
  *     per device, with that device current); make that first call before any
  *     stream capture on that device.

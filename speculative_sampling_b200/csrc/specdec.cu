@@ -40,6 +40,7 @@
 #include <climits>
 #include <cstring>
 #include <mutex>
+#include <string>
 #include <unordered_map>
 #include <vector>
 
@@ -59,13 +60,6 @@ struct __align__(16) Partial {  // one (row, V-split): max and sum of 2^((z-m)c)
   double s;
   float m;
   uint32_t pad;
-};
-struct __align__(16) Sel {  // per sequence: what the draw needs
-  double St, Sd;            // normalisers of the drawn target/draft rows
-  double c64;               // log2(e) / T
-  float Mt, Md;             // maxima of the drawn rows
-  int n;                    // draw position (= accepted count), -1 if invalid
-  int pad;
 };
 struct __align__(16) ResPartial {  // one (sequence, V-chunk) of the drawn row(s)
   double R;                        // sum of St * max(0, p - q)  (or of 2^((z-m)c), bonus)
@@ -107,20 +101,6 @@ __device__ __forceinline__ float fmax_nan(float a, float b) {
   return y;
 }
 
-__device__ __forceinline__ uint4 ld_stream(const uint4 *p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-
-__device__ __forceinline__ __nv_bfloat162 as_bf162(uint32_t w) {
-  __nv_bfloat162 v;
-  memcpy(&v, &w, sizeof v);
-  return v;
-}
-
 template <typename T>
 struct Dt;
 template <>
@@ -141,18 +121,6 @@ struct Dt<__nv_bfloat16> {
       x[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
     }
   }
-  template <int U>
-  static __device__ __forceinline__ float tile_max(const uint4 (&buf)[U]) {
-    __nv_bfloat162 mx = as_bf162(buf[0].x);
-#pragma unroll
-    for (int k = 0; k < U; ++k) {
-      const uint32_t w[4] = {buf[k].x, buf[k].y, buf[k].z, buf[k].w};
-#pragma unroll
-      for (int q = (k == 0 ? 1 : 0); q < 4; ++q)
-        mx = __hmax2_nan(mx, as_bf162(w[q]));
-    }
-    return fmax_nan(__low2float(mx), __high2float(mx));
-  }
 };
 template <>
 struct Dt<float> {
@@ -166,18 +134,6 @@ struct Dt<float> {
     x[1] = __uint_as_float(v.y);
     x[2] = __uint_as_float(v.z);
     x[3] = __uint_as_float(v.w);
-  }
-  template <int U>
-  static __device__ __forceinline__ float tile_max(const uint4 (&buf)[U]) {
-    float m = __uint_as_float(buf[0].x);
-#pragma unroll
-    for (int k = 0; k < U; ++k) {
-      float x[4];
-      unpack(buf[k], x);
-#pragma unroll
-      for (int q = (k == 0 ? 1 : 0); q < 4; ++q) m = fmax_nan(m, x[q]);
-    }
-    return m;
   }
 };
 
@@ -201,38 +157,6 @@ __device__ __forceinline__ void online_add(float &m, float &s, float x, Scale c)
   }
 }
 
-// Fold one register tile (U vectors per thread) into (m, s).
-template <typename T, int U>
-__device__ __forceinline__ void tile_update(const uint4 (&buf)[U], float &m, float &s, Scale c) {
-  constexpr int VEC = Dt<T>::VEC;
-  const float tmax = Dt<T>::template tile_max<U>(buf);
-  if (!(tmax <= m)) {  // new max (or NaN): rescale what we have
-    s = s * ex2(scaled(m - tmax, c));
-    m = tmax;
-  }
-  if (m != -INFINITY) {
-    float vs[U];
-#pragma unroll
-    for (int k = 0; k < U; ++k) {
-      float x[VEC];
-      Dt<T>::unpack(buf[k], x);
-      float e[VEC];
-#pragma unroll
-      for (int q = 0; q < VEC; ++q) e[q] = ex2(scaled(x[q] - m, c));
-#pragma unroll
-      for (int w = 1; w < VEC; w *= 2)  // pairwise tree within the vector
-#pragma unroll
-        for (int q = 0; q < VEC; q += 2 * w) e[q] += e[q + w];
-      vs[k] = e[0];
-    }
-#pragma unroll
-    for (int w = 1; w < U; w *= 2)
-#pragma unroll
-      for (int k = 0; k + w < U; k += 2 * w) vs[k] += vs[k + w];
-    s += vs[0];
-  }
-}
-
 __device__ __forceinline__ double warp_sum(double v) {
 #pragma unroll
   for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
@@ -244,198 +168,348 @@ __device__ __forceinline__ float warp_max_nan(float v) {
   return v;
 }
 
-// Combine per-thread (m, s) over the CTA: returns (M, S) in thread 0.
-__device__ __forceinline__ void block_combine(float m, float s, Scale c, float &M, double &S) {
-  __shared__ float sm_m[NWARP];
-  __shared__ double sm_s[NWARP];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const float mw = warp_max_nan(m);
-  double sl = (m == -INFINITY) ? 0.0 : (double)s * (double)ex2(scaled(m - mw, c));
-  sl = warp_sum(sl);
-  if (lane == 0) {
-    sm_m[warp] = mw;
-    sm_s[warp] = sl;
+// ---------------------------------------------------------------------------
+// kernel 1: softmax statistics of every row
+// ---------------------------------------------------------------------------
+// The B*(2K+1) rows are cut into units: a unit is UT consecutive tiles of one
+// row; a tile is CW*32*U 16-byte vectors (16 KB for U = 4).  CTA g of a grid
+// of G handles units g, g+G, g+2G, ... so the grid sweeps the logits front to
+// back, sequence after sequence.
+//
+// Warp specialisation: one producer warp streams tiles with cp.async.bulk
+// (the TMA bulk-copy engine; plain CTA-local copies, no multicast) into an
+// NSTAGE-deep ring in shared memory, tracked by "full" / "empty" mbarriers;
+// CW consumer warps take a tile out of the ring (one 16-byte shared load per
+// vector), release the slot, and fold it into a per-thread (max, sum) in
+// registers.  A unit's setup (row pointer, alignment, log2(e)/T) and its
+// CTA combine are paid once per unit.  Per element the consumers spend one
+// exact bf16->fp32 unpack, one FMNMX for the tile max, three packed fp32x2
+// operations at half an issue slot each, one MUFU ex2 and half a packed add.
+// Every wait is bounded: a wait that runs out sets SPECDEC_ERR_TIMEOUT in the
+// device error word and the kernel winds down (the producer first waits, again
+// bounded, for the copies it has in flight).
+
+constexpr int CW = 8;               // consumer warps
+constexpr int NTC = CW * 32;        // consumer threads
+constexpr int NTS = NTC + 32;       // + one producer warp
+constexpr int NSTAGE = 3;           // depth of the shared-memory ring
+constexpr unsigned kWaitLimit = 1u << 22;  // try_wait rounds before giving up
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t *bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_tx(uint64_t *bar, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, unsigned parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// bounded wait for the phase of the given parity; false when it ran out
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, unsigned parity) {
+  for (unsigned i = 0; i < kWaitLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  atomicOr(&g_error_flags, SPECDEC_ERR_TIMEOUT);
+  return false;
+}
+// global -> shared bulk copy completing on an mbarrier (16-byte aligned
+// addresses, size a multiple of 16)
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, unsigned bytes,
+                                          uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ uint4 lds128(const void *p) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(smem_u32(p)));
+  return v;
+}
+// pairs (x0, x1) of the 8 (bf16) or 4 (fp32) values of a 16-byte vector
+template <typename T>
+struct Pairs;
+template <>
+struct Pairs<__nv_bfloat16> {
+  static constexpr int N = 4;
+  static __device__ __forceinline__ float2 get(const uint4 &v, int q) {
+    const uint32_t w = q == 0 ? v.x : q == 1 ? v.y : q == 2 ? v.z : v.w;
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+  }
+};
+template <>
+struct Pairs<float> {
+  static constexpr int N = 2;
+  static __device__ __forceinline__ float2 get(const uint4 &v, int q) {
+    return q == 0 ? make_float2(__uint_as_float(v.x), __uint_as_float(v.y))
+                  : make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
+  }
+};
+
+// Fold one 16-byte vector into the thread's (m, s): the vector's max by a
+// depth-3 FMNMX tree (NaN propagating), a rescale of s when the running max
+// grows, then packed fp32x2 exponent arguments, MUFU ex2 and a pairwise
+// packed sum.  Only the vector's 8 (bf16) or 4 (fp32) values are live.
+template <typename T>
+__device__ __forceinline__ void vec_fold(const uint4 &v, float &m, float &s, Scale c) {
+  constexpr int N = Pairs<T>::N;
+  float2 x[N];
+#pragma unroll
+  for (int q = 0; q < N; ++q) x[q] = Pairs<T>::get(v, q);
+  float mx[N];
+#pragma unroll
+  for (int q = 0; q < N; ++q) mx[q] = fmax_nan(x[q].x, x[q].y);
+#pragma unroll
+  for (int w = 1; w < N; w *= 2)
+#pragma unroll
+    for (int q = 0; q + w < N; q += 2 * w) mx[q] = fmax_nan(mx[q], mx[q + w]);
+  if (!(mx[0] <= m)) {  // new running max (or NaN): rescale what we have
+    s = s * ex2(scaled(m - mx[0], c));
+    m = mx[0];
+  }
+  if (m != -INFINITY) {
+    const float2 nm = make_float2(-m, -m), hi = make_float2(c.hi, c.hi),
+                 lo = make_float2(c.lo, c.lo);
+    float2 e[N];
+#pragma unroll
+    for (int q = 0; q < N; ++q) {
+      const float2 d = __fadd2_rn(x[q], nm);
+      const float2 a = __ffma2_rn(d, hi, __fmul2_rn(d, lo));
+      e[q] = make_float2(ex2(a.x), ex2(a.y));
+    }
+#pragma unroll
+    for (int w = 1; w < N; w *= 2)
+#pragma unroll
+      for (int q = 0; q + w < N; q += 2 * w) e[q] = __fadd2_rn(e[q], e[q + w]);
+    s += e[0].x + e[0].y;
+  }
+}
+
+struct StatsGeom {
+  int K;
+  long long V;
+  int tpr;          // tiles per row
+  long long tiles;  // rows * tpr
+  int slots;        // CTA slots per row (>= CTAs that can share one row)
+};
+
+// CTA g of G owns tiles [g*T/G, (g+1)*T/G); the owner of tile t is then
+// floor(((t+1)*G - 1) / T).  Both the statistics kernel and the combine in
+// k_finish use these to name a row's partials: CTA slot = owner - first owner,
+// and each of the CW consumer warps of a CTA writes its own partial.
+__host__ __device__ __forceinline__ long long tile_begin(long long g, long long G, long long T) {
+  return g * T / G;
+}
+__host__ __device__ __forceinline__ long long tile_owner(long long t, long long G, long long T) {
+  return ((t + 1) * G - 1) / T;
+}
+
+// The current row of a CTA's tile walk.  Rows are numbered b*(2K+1) + j with
+// j = 0..K the target rows and j = K+1..2K the draft rows of sequence b; the
+// cursor steps row by row without divisions.
+template <typename T>
+struct RowCursor {
+  const T *p;
+  const uint4 *pv;
+  long long row, b, nvec;
+  int j, ti, head;
+  __device__ __forceinline__ void point(const T *target, const T *draft, const StatsGeom &g) {
+    constexpr int VEC = Dt<T>::VEC;
+    p = (j <= g.K) ? target + (b * (g.K + 1) + j) * g.V
+                   : draft + (b * g.K + (j - g.K - 1)) * g.V;
+    head = row_head(p, g.V);
+    nvec = (g.V - head) / VEC;
+    pv = reinterpret_cast<const uint4 *>(p + head);
+  }
+  __device__ __forceinline__ void start(const T *target, const T *draft, const StatsGeom &g,
+                                        long long t) {
+    const int R = 2 * g.K + 1;
+    row = t / g.tpr;
+    ti = (int)(t - row * g.tpr);
+    b = row / R;
+    j = (int)(row - b * R);
+    point(target, draft, g);
+  }
+  __device__ __forceinline__ void next_row(const T *target, const T *draft, const StatsGeom &g) {
+    ++row;
+    ti = 0;
+    if (++j == 2 * g.K + 1) {
+      j = 0;
+      ++b;
+    }
+    point(target, draft, g);
+  }
+};
+
+template <typename T, int U>
+__global__ void __launch_bounds__(NTS) k_row_stats(const T *__restrict__ target,
+                                                   const T *__restrict__ draft,
+                                                   const float *__restrict__ temperature,
+                                                   StatsGeom g, Partial *__restrict__ part,
+                                                   unsigned *__restrict__ tickets, int B) {
+  constexpr int VEC = Dt<T>::VEC;
+  constexpr long long TV = (long long)NTC * U;  // vectors per tile
+  constexpr unsigned TILE_BYTES = (unsigned)TV * 16u;
+  extern __shared__ __align__(128) unsigned char ring[];  // NSTAGE * TILE_BYTES
+  __shared__ __align__(8) uint64_t full[NSTAGE], empty[NSTAGE];
+  __shared__ int s_abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long G = gridDim.x;
+  const long long t0 = tile_begin(blockIdx.x, G, g.tiles);
+  const long long t1 = tile_begin(blockIdx.x + 1, G, g.tiles);
+
+  // the arrival tickets of k_finish (which runs after this kernel) start at 0
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < B; i += blockDim.x) tickets[i] = 0u;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NSTAGE; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], CW);
+    }
+    s_abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  if (warp == 0) {
-    const float m2 = lane < NWARP ? sm_m[lane] : -INFINITY;
-    const double s2 = lane < NWARP ? sm_s[lane] : 0.0;
-    const float mb = warp_max_nan(m2);
-    double f = (m2 == -INFINITY) ? 0.0 : s2 * (double)ex2(scaled(m2 - mb, c));
-    f = warp_sum(f);
-    M = mb;
-    S = f;
+  if (t0 >= t1) return;
+
+  if (warp == CW) {  // ---------------- producer warp ----------------
+    if (lane != 0) return;
+    unsigned it = 0;
+    RowCursor<T> rc;
+    rc.start(target, draft, g, t0);
+    for (long long t = t0; t < t1 && !*(volatile int *)&s_abort; ++t) {
+      if (rc.ti == g.tpr) rc.next_row(target, draft, g);
+      const long long v0 = (long long)rc.ti * TV;
+      const long long v1 = (v0 + TV < rc.nvec) ? v0 + TV : rc.nvec;
+      ++rc.ti;
+      if (v0 >= v1) continue;  // an empty last tile (the row's tail is scalar)
+      const int st = (int)(it % NSTAGE);
+      if (!mbar_wait(&empty[st], ((it / NSTAGE) & 1u) ^ 1u)) {
+        atomicExch(&s_abort, 1);
+        break;
+      }
+      const unsigned bytes = (unsigned)(v1 - v0) * 16u;
+      mbar_arrive_tx(&full[st], bytes);
+      bulk_load(ring + (size_t)st * TILE_BYTES, rc.pv + v0, bytes, &full[st]);
+      ++it;
+    }
+    // The CTA must not retire with copies in flight: wait (bounded) until the
+    // last copy issued into each slot has landed.
+    for (unsigned k = 0; k < NSTAGE && k < it; ++k) {
+      const unsigned j = it - 1 - k;
+      mbar_wait(&full[j % NSTAGE], (j / NSTAGE) & 1u);
+    }
+    return;
   }
-}
 
-// ---------------------------------------------------------------------------
-// kernel 1: per-(row, V-split) softmax statistics
-// ---------------------------------------------------------------------------
-template <typename T, int U>
-__global__ void __launch_bounds__(NT) k_row_stats(const T *__restrict__ target,
-                                                  const T *__restrict__ draft,
-                                                  const float *__restrict__ temperature, int K,
-                                                  long long V, int nsplit,
-                                                  Partial *__restrict__ part) {
-  constexpr int VEC = Dt<T>::VEC;
-  const int R = 2 * K + 1;
-  const long long row = (long long)blockIdx.x / nsplit;
-  const int split = (int)((long long)blockIdx.x - row * nsplit);
-  const long long b = row / R;
-  const int j = (int)(row - b * R);
-  const T *p = (j <= K) ? target + (b * (K + 1) + j) * V : draft + (b * K + (j - K - 1)) * V;
-  const Scale c = make_scale(kLog2e / (double)temperature[b]);
-
-  const int head = row_head(p, V);
-  const long long nvec = (V - head) / VEC;
-  const uint4 *pv = reinterpret_cast<const uint4 *>(p + head);
-  const long long v0 = (long long)split * (NT * U) + threadIdx.x;
-
-  uint4 buf[U];
-#pragma unroll
-  for (int k = 0; k < U; ++k) {
-    const long long vi = v0 + (long long)k * NT;
-    buf[k] = (vi < nvec) ? ld_stream(pv + vi) : Dt<T>::neg_inf();
-  }
+  // ---------------- consumer warps ----------------
+  // No CTA-wide barrier inside the walk: each warp folds its share of every
+  // tile and, at the end of a row (or of the CTA's range), reduces its lanes
+  // and writes its own partial.  After an abort the waits and the arithmetic
+  // are skipped.
+  unsigned it = 0;
+  RowCursor<T> rc;
+  rc.start(target, draft, g, t0);
+  Scale c = make_scale(kLog2e / (double)__ldg(temperature + rc.b));
+  // temperature of the sequence after this one, fetched a row ahead
+  float T_next = (rc.b + 1 < B) ? __ldg(temperature + rc.b + 1) : 1.0f;
   float m = -INFINITY, s = 0.0f;
-  tile_update<T, U>(buf, m, s, c);
-  if (split == 0 && (int)threadIdx.x < head) online_add(m, s, Dt<T>::load(p + threadIdx.x), c);
-  if (split == nsplit - 1) {
-    const long long t = head + nvec * VEC + threadIdx.x;
-    if (t < V) online_add(m, s, Dt<T>::load(p + t), c);
-  }
-  float M;
-  double S;
-  block_combine(m, s, c, M, S);
-  if (threadIdx.x == 0) {
-    Partial out;
-    out.s = S;
-    out.m = M;
-    out.pad = 0;
-    part[row * nsplit + split] = out;
-  }
-}
-
-// ---------------------------------------------------------------------------
-// kernel 2: combine, gather p(x), q(x), accept test, first rejection
-// ---------------------------------------------------------------------------
-template <typename T>
-__global__ void __launch_bounds__(128) k_accept(
-    const T *__restrict__ target, const T *__restrict__ draft,
-    const int32_t *__restrict__ tokens, const float *__restrict__ u_accept,
-    const float *__restrict__ temperature, int B, int K, long long V, int nsplit,
-    const Partial *__restrict__ part, Sel *__restrict__ sel, unsigned *__restrict__ counters,
-    int32_t *__restrict__ out_tokens, int32_t *__restrict__ out_n,
-    float *__restrict__ dbg_row_max, double *__restrict__ dbg_row_sum,
-    double *__restrict__ dbg_px, double *__restrict__ dbg_qx) {
-  const int lane = threadIdx.x & 31;
-  const long long b = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
-  if (b >= B) return;
-  const int R = 2 * K + 1;
-  const float Tf = temperature[b];
-  const bool t_ok = isfinite(Tf) && Tf > 0.0f;
-  const double c64 = kLog2e / (double)Tf;
-
-  // combine the V-splits of every row in fp64; lane i keeps the statistics of
-  // target row i and draft row i, every lane keeps those of target row K
-  float my_mt = 0.f, my_md = 0.f, mk = 0.f;
-  double my_st = 1.0, my_sd = 1.0, sk = 1.0;
-  bool rows_ok = true;
-  for (int r = 0; r < R; ++r) {
-    const Partial *P = part + (b * R + r) * nsplit;
-    float m = -INFINITY;
-    for (int s = lane; s < nsplit; s += 32) m = fmaxf(m, P[s].m);
-    m = warp_max_nan(m);
-    double acc = 0.0;
-    for (int s = lane; s < nsplit; s += 32) {
-      const Partial ps = P[s];
-      acc += (ps.m == -INFINITY) ? ps.s : ps.s * exp2(((double)ps.m - (double)m) * c64);
+  int seg_first = rc.ti;  // first tile of this row in this CTA's range
+  for (long long t = t0; t < t1; ++t) {
+    const long long v0 = (long long)rc.ti * TV;
+    const long long v1 = (v0 + TV < rc.nvec) ? v0 + TV : rc.nvec;
+    if (v0 < v1) {
+      const int st = (int)(it % NSTAGE);
+      bool have = false;
+      if (!*(volatile int *)&s_abort) {
+        have = __all_sync(FULL, mbar_wait(&full[st], (it / NSTAGE) & 1u));
+        if (!have && lane == 0) atomicExch(&s_abort, 1);
+      }
+      ++it;
+      if (have) {
+        const long long nv = v1 - v0;
+        const unsigned char *tile = ring + (size_t)st * TILE_BYTES;
+        uint4 v[U];
+#pragma unroll
+        for (int k = 0; k < U; ++k) {
+          const int vi = k * NTC + threadIdx.x;
+          v[k] = (vi < nv) ? lds128(tile + (size_t)vi * 16) : Dt<T>::neg_inf();
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
+#pragma unroll
+        for (int k = 0; k < U; ++k) vec_fold<T>(v[k], m, s, c);
+      }
     }
-    acc = warp_sum(acc);
-    rows_ok = rows_ok && isfinite(m) && isfinite(acc) && acc > 0.0;
-    if (r < K && lane == r) {
-      my_mt = m;
-      my_st = acc;
-    } else if (r == K) {
-      mk = m;
-      sk = acc;
-    } else if (r > K && lane == r - K - 1) {
-      my_md = m;
-      my_sd = acc;
-    }
-    if (lane == 0) {
-      if (dbg_row_max) dbg_row_max[b * R + r] = m;
-      if (dbg_row_sum) dbg_row_sum[b * R + r] = acc;
-    }
-  }
-
-  // gather and test, one draft position per lane
-  int x = 0;
-  bool x_ok = true, acc_i = false;
-  double p = 0.0, q = 0.0;
-  if (lane < K) {
-    x = tokens[b * K + lane];
-    x_ok = (x >= 0) && ((long long)x < V);
-    if (x_ok && rows_ok && t_ok) {
-      const float zt = Dt<T>::load(target + (b * (K + 1) + lane) * V + x);
-      const float zd = Dt<T>::load(draft + (b * K + lane) * V + x);
-      p = exp2(((double)zt - (double)my_mt) * c64) / my_st;
-      q = exp2(((double)zd - (double)my_md) * c64) / my_sd;
-      acc_i = (double)u_accept[b * K + lane] * q < p;
-    }
-  }
-  const unsigned bad_x = __ballot_sync(FULL, lane < K && !x_ok);
-  const unsigned accm = __ballot_sync(FULL, lane < K && acc_i);
-  const bool seq_ok = t_ok && rows_ok && bad_x == 0;
-  const unsigned kmask = (K >= 32) ? FULL : ((1u << K) - 1u);
-  const unsigned rej = ~accm & kmask;
-  const int n = seq_ok ? (rej ? __ffs(rej) - 1 : K) : -1;
-
-  int32_t *ot = out_tokens + b * (K + 1);
-  if (!seq_ok) {
-    for (int i = lane; i <= K; i += 32) ot[i] = -1;
-  } else {
-    if (lane < n) ot[lane] = x;
-    for (int i = n + 1 + lane; i <= K; i += 32) ot[i] = -1;
-    if (lane < K && lane <= n) {
-      if (dbg_px) dbg_px[b * K + lane] = p;
-      if (dbg_qx) dbg_qx[b * K + lane] = q;
-    }
-  }
-  // the lane holding the drawn row's statistics publishes them
-  const int owner = (seq_ok && n < K) ? n : 0;
-  if (lane == owner) {
-    Sel o;
-    o.n = n;
-    o.pad = 0;
-    o.c64 = c64;
-    if (seq_ok && n < K) {
-      o.Mt = my_mt;
-      o.St = my_st;
-      o.Md = my_md;
-      o.Sd = my_sd;
-    } else {
-      o.Mt = mk;
-      o.St = sk;
-      o.Md = 0.f;
-      o.Sd = 1.0;
-    }
-    sel[b] = o;
-    counters[b] = 0;  // arrival ticket of k_resample for this sequence
-    out_n[b] = n;
-    if (!seq_ok) {
-      unsigned f = 0;
-      if (!t_ok) f |= SPECDEC_ERR_TEMPERATURE;
-      if (bad_x) f |= SPECDEC_ERR_TOKEN;
-      if (!rows_ok) f |= SPECDEC_ERR_LOGITS;
-      atomicOr(&g_error_flags, f);
+    ++rc.ti;
+    if (rc.ti == g.tpr || t + 1 == t1) {  // end of this CTA's part of the row
+      // scalar head / tail of the row when this CTA holds its first / last tile
+      if (seg_first == 0 && (int)threadIdx.x < rc.head)
+        online_add(m, s, Dt<T>::load(rc.p + threadIdx.x), c);
+      if (rc.ti == g.tpr) {
+        const long long tt = rc.head + rc.nvec * VEC + threadIdx.x;
+        if (tt < g.V) online_add(m, s, Dt<T>::load(rc.p + tt), c);
+      }
+      // this warp's partial: lanes combined in fp64 with shuffles
+      const float mw = warp_max_nan(m);
+      double sw = (m == -INFINITY) ? 0.0 : (double)s * (double)ex2(scaled(m - mw, c));
+      sw = warp_sum(sw);
+      if (lane == 0) {
+        const long long slot = (long long)blockIdx.x - tile_owner(rc.row * g.tpr, G, g.tiles);
+        Partial out;
+        out.s = sw;
+        out.m = mw;
+        out.pad = 0;
+        part[(rc.row * g.slots + slot) * CW + warp] = out;
+      }
+      if (t + 1 < t1) {  // next row
+        const bool new_seq = (rc.j == 2 * g.K);
+        rc.next_row(target, draft, g);
+        if (new_seq) {
+          c = make_scale(kLog2e / (double)T_next);
+          T_next = (rc.b + 1 < B) ? __ldg(temperature + rc.b + 1) : 1.0f;
+        }
+        m = -INFINITY;
+        s = 0.0f;
+        seg_first = 0;
+      }
     }
   }
 }
 
 // ---------------------------------------------------------------------------
-// kernel 3: residual / bonus draw
+// kernel 2: accept test + residual / bonus draw ("finish")
 // ---------------------------------------------------------------------------
+// Grid: B sequences x nsr V-chunks.  Every CTA of sequence b first repeats the
+// (small) acceptance step for b: it combines the V-split partials of the 2K+1
+// rows in fp64, gathers p_i(x_i) and q_i(x_i) (fp64 exp2 of exact logits),
+// tests u*q < p on K lanes and finds the first rejection n with __ballot_sync /
+// __ffs.  Chunk 0 writes the accepted prefix.  Then each CTA streams its chunk
+// of the drawn row pair (target/draft row n, or the target's row K for the
+// bonus), forming r(v) = St * max(0, p - q) = max(0, e_t - (St/Sd) e_d) on the
+// fly (or e_t for the bonus), and adds it up in fp64.  The last CTA of the
+// sequence to finish (atomic arrival ticket; nothing waits) draws: block scan
+// of the chunk sums in fp64, the chunk holding u*Z, then a block scan over
+// that chunk with the weights kept in registers, first crossing wins.  When
+// the residual mass is below 2^-64 the fp32 weights have run out of range and
+// the draw is redone in fp64 over the whole row pair.
+
 struct DrawRow {
   float Mt, Md, lhi, llo;
   Scale c;
@@ -490,15 +564,16 @@ __device__ __forceinline__ double prob64(const T *row, long long v, float M, dou
 // residual is zero as well, draws from p (as the oracle does).  Used only when
 // the fp32 residual weights have run out of range.
 template <typename T>
-__device__ __noinline__ int draw_exact64(const T *pt, const T *pd, long long V, const Sel &sl, double u,
-                            int *s_y, int *s_lastpos, double *dbg_Z) {
+__device__ __noinline__ int draw_exact64(const T *pt, const T *pd, long long V, float Mt,
+                                         double St, float Md, double Sd, double c64, double u,
+                                         int *s_y, int *s_lastpos, double *dbg_Z) {
   const long long E = (V + NT - 1) / NT;
   const long long e0 = (long long)threadIdx.x * E < V ? (long long)threadIdx.x * E : V;
   const long long e1 = (e0 + E < V) ? e0 + E : V;
   double sr = 0.0, sp = 0.0;
   for (long long v = e0; v < e1; ++v) {
-    const double p = prob64(pt, v, sl.Mt, sl.St, sl.c64);
-    const double q = prob64(pd, v, sl.Md, sl.Sd, sl.c64);
+    const double p = prob64(pt, v, Mt, St, c64);
+    const double q = prob64(pd, v, Md, Sd, c64);
     sr += (p - q > 0.0) ? p - q : 0.0;
     sp += p;
   }
@@ -512,8 +587,8 @@ __device__ __noinline__ int draw_exact64(const T *pt, const T *pd, long long V, 
   int last = -1;
   bool found = false;
   for (long long v = e0; v < e1; ++v) {
-    const double p = prob64(pt, v, sl.Mt, sl.St, sl.c64);
-    const double q = prob64(pd, v, sl.Md, sl.Sd, sl.c64);
+    const double p = prob64(pt, v, Mt, St, c64);
+    const double q = prob64(pd, v, Md, Sd, c64);
     const double x = use_p ? p : ((p - q > 0.0) ? p - q : 0.0);
     if (x > 0.0) last = (int)v;
     C += x;
@@ -530,33 +605,143 @@ __device__ __noinline__ int draw_exact64(const T *pt, const T *pd, long long V, 
 }
 
 template <typename T, int UR>
-__global__ void __launch_bounds__(NT) k_resample(
+__global__ void __launch_bounds__(NT) k_finish(
     const T *__restrict__ target, const T *__restrict__ draft,
-    const float *__restrict__ u_resample, int K, long long V, int nsr,
-    const Sel *__restrict__ sel, ResPartial *__restrict__ rpart, unsigned *__restrict__ counters,
-    int32_t *__restrict__ out_tokens, double *__restrict__ dbg_Z) {
+    const int32_t *__restrict__ tokens, const float *__restrict__ u_accept,
+    const float *__restrict__ u_resample, const float *__restrict__ temperature, int K,
+    long long V, int tpr, long long tiles, long long G1, int slots, int nsr,
+    const Partial *__restrict__ part,
+    ResPartial *__restrict__ rpart, unsigned *__restrict__ counters,
+    int32_t *__restrict__ out_tokens, int32_t *__restrict__ out_n,
+    float *__restrict__ dbg_row_max, double *__restrict__ dbg_row_sum,
+    double *__restrict__ dbg_px, double *__restrict__ dbg_qx, double *__restrict__ dbg_Z) {
   constexpr int VEC = Dt<T>::VEC;
   constexpr long long CH = (long long)NT * UR * VEC;  // elements per chunk
+  constexpr int EMAX = UR * VEC + 1;                  // rescan elements per thread
+  __shared__ float sM[65];
+  __shared__ double sS[65];
+  __shared__ int s_n, s_last, s_mode, s_chunk, s_y, s_lastpos;
+  __shared__ double s_base, s_t;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const long long b = (long long)blockIdx.x / nsr;
   const int chunk = (int)((long long)blockIdx.x - b * nsr);
-  const Sel sl = sel[b];
-  if (sl.n < 0) return;  // invalid sequence: the accept kernel wrote its outputs
+  const int R = 2 * K + 1;
+
+  // ---- inputs of this call (independent of the statistics kernel) ----
+  const float Tf = __ldg(temperature + b);
+  const bool t_ok = isfinite(Tf) && Tf > 0.0f;
+  const double c64 = kLog2e / (double)Tf;
+  int x = 0;
+  bool x_ok = true;
+  float zt_x = 0.f, zd_x = 0.f, u = 0.f;
+  if (warp == 0 && lane < K) {
+    x = __ldg(tokens + b * K + lane);
+    x_ok = (x >= 0) && ((long long)x < V);
+    u = __ldg(u_accept + b * K + lane);
+    if (x_ok) {
+      zt_x = Dt<T>::load(target + (b * (K + 1) + lane) * V + x);
+      zd_x = Dt<T>::load(draft + (b * K + lane) * V + x);
+    }
+  }
+  const float ures = __ldg(u_resample + b);
+  cudaGridDependencySynchronize();  // the row statistics are complete from here on
+
+  // ---- combine the V-split partials of every row (fp64) ----
+  for (int r = warp; r < R; r += NWARP) {
+    const long long row = b * R + r;
+    const Partial *P = part + row * slots * CW;
+    // partials of the CTAs of the statistics sweep that hold tiles of this
+    // row, in order, CW consumer warps each
+    const int nslot = (int)(tile_owner(row * tpr + tpr - 1, G1, tiles) -
+                            tile_owner(row * tpr, G1, tiles) + 1) * CW;
+    float m = -INFINITY;
+    for (int s = lane; s < nslot; s += 32) m = fmaxf(m, P[s].m);
+    m = warp_max_nan(m);
+    double acc = 0.0;
+    for (int s = lane; s < nslot; s += 32) {
+      const Partial ps = P[s];
+      acc += (ps.m == -INFINITY) ? ps.s : ps.s * exp2(((double)ps.m - (double)m) * c64);
+    }
+    acc = warp_sum(acc);
+    if (lane == 0) {
+      sM[r] = m;
+      sS[r] = acc;
+      if (chunk == 0 && dbg_row_max) dbg_row_max[b * R + r] = m;
+      if (chunk == 0 && dbg_row_sum) dbg_row_sum[b * R + r] = acc;
+    }
+  }
+  __syncthreads();
+
+  // ---- acceptance test and first rejection (warp 0) ----
+  if (warp == 0) {
+    // a timed-out wait in this call (or an earlier, unacknowledged one) makes
+    // every sequence invalid rather than silently wrong
+    const bool timed_out = (*(volatile unsigned *)&g_error_flags & SPECDEC_ERR_TIMEOUT) != 0;
+    bool rows_ok = true;
+    for (int r = lane; r < R; r += 32)
+      rows_ok = rows_ok && isfinite(sM[r]) && isfinite(sS[r]) && sS[r] > 0.0;
+    rows_ok = __all_sync(FULL, rows_ok) && !timed_out;
+    bool acc_i = false;
+    double p = 0.0, q = 0.0;
+    if (lane < K && x_ok && rows_ok && t_ok) {
+      p = exp2(((double)zt_x - (double)sM[lane]) * c64) / sS[lane];
+      q = exp2(((double)zd_x - (double)sM[K + 1 + lane]) * c64) / sS[K + 1 + lane];
+      acc_i = (double)u * q < p;
+    }
+    const unsigned bad_x = __ballot_sync(FULL, lane < K && !x_ok);
+    const unsigned accm = __ballot_sync(FULL, lane < K && acc_i);
+    const bool seq_ok = t_ok && rows_ok && bad_x == 0;
+    const unsigned kmask = (K >= 32) ? FULL : ((1u << K) - 1u);
+    const unsigned rej = ~accm & kmask;
+    const int n = seq_ok ? (rej ? __ffs(rej) - 1 : K) : -1;
+    if (lane == 0) s_n = n;
+    if (chunk == 0) {
+      int32_t *ot = out_tokens + b * (K + 1);
+      if (!seq_ok) {
+        for (int i = lane; i <= K; i += 32) ot[i] = -1;
+      } else {
+        if (lane < n) ot[lane] = x;
+        for (int i = n + 1 + lane; i <= K; i += 32) ot[i] = -1;
+        if (lane < K && lane <= n) {
+          if (dbg_px) dbg_px[b * K + lane] = p;
+          if (dbg_qx) dbg_qx[b * K + lane] = q;
+        }
+      }
+      if (lane == 0) {
+        out_n[b] = n;
+        if (!seq_ok) {
+          unsigned f = 0;
+          if (!t_ok) f |= SPECDEC_ERR_TEMPERATURE;
+          if (bad_x) f |= SPECDEC_ERR_TOKEN;
+          if (!rows_ok) f |= SPECDEC_ERR_LOGITS;
+          atomicOr(&g_error_flags, f);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  const int n = s_n;
+  if (n < 0) return;  // invalid sequence (the same for every CTA of it)
+
+  // ---- this CTA's chunk of the drawn row pair ----
   DrawRow d;
-  d.bonus = (sl.n == K);
-  d.Mt = sl.Mt;
-  d.Md = sl.Md;
-  d.c = make_scale(sl.c64);
-  const double lam = d.bonus ? 0.0 : sl.St / sl.Sd;
+  d.bonus = (n == K);
+  d.Mt = sM[n];
+  const double St = sS[n];
+  d.Md = d.bonus ? 0.f : sM[K + 1 + n];
+  const double Sd = d.bonus ? 1.0 : sS[K + 1 + n];
+  d.c = make_scale(c64);
+  const double lam = d.bonus ? 0.0 : St / Sd;
   d.lhi = (float)lam;
   d.llo = (float)(lam - (double)d.lhi);
-  const T *pt = target + (b * (K + 1) + sl.n) * V;
-  const T *pd = d.bonus ? pt : draft + (b * K + sl.n) * V;
+  const T *pt = target + (b * (K + 1) + n) * V;
+  const T *pd = d.bonus ? pt : draft + (b * K + n) * V;
 
   const int head = row_head(pt, V);
   const bool vec_ok = row_head(pd, V) == head;
   const long long nvec = vec_ok ? (V - head) / VEC : 0;
-  // chunk c covers elements [lo_c, hi_c): chunk 0 also takes the head, the
-  // last chunk also takes the tail
+  // chunk c covers elements [lo_c, hi_c): chunk 0 also takes the head, and the
+  // chunk whose range holds the < VEC tail elements takes those
   auto chunk_lo = [&](int cidx) -> long long {
     if (cidx == 0) return 0;
     const long long v = head + (long long)cidx * CH;
@@ -572,19 +757,24 @@ __global__ void __launch_bounds__(NT) k_resample(
   if (vec_ok) {
     const uint4 *vt = reinterpret_cast<const uint4 *>(pt + head);
     const uint4 *vd = reinterpret_cast<const uint4 *>(pd + head);
+    uint4 at[UR], ad[UR];
+#pragma unroll
+    for (int k = 0; k < UR; ++k) {
+      const long long vi = (long long)chunk * NT * UR + (long long)k * NT + threadIdx.x;
+      at[k] = vi < nvec ? __ldg(vt + vi) : make_uint4(0, 0, 0, 0);
+      ad[k] = (vi < nvec && !d.bonus) ? __ldg(vd + vi) : make_uint4(0, 0, 0, 0);
+    }
 #pragma unroll
     for (int k = 0; k < UR; ++k) {
       const long long vi = (long long)chunk * NT * UR + (long long)k * NT + threadIdx.x;
       if (vi < nvec) {
-        float xt[VEC], xd[VEC] = {};
-        Dt<T>::unpack(ld_stream(vt + vi), xt);
-        if (!d.bonus) Dt<T>::unpack(ld_stream(vd + vi), xd);
+        float xt[VEC], xd[VEC];
+        Dt<T>::unpack(at[k], xt);
+        Dt<T>::unpack(ad[k], xd);
 #pragma unroll
-        for (int q = 0; q < VEC; ++q) rs += res_weight(xt[q], d.bonus ? 0.f : xd[q], d);
+        for (int q = 0; q < VEC; ++q) rs += res_weight(xt[q], xd[q], d);
       }
     }
-    // head elements belong to chunk 0; the < VEC tail elements to the chunk
-    // whose element range [lo_c, hi_c) holds them (the rescan uses the same)
     // (a thread may own one head and one tail element of the same chunk)
     const long long tail_chunk = nvec / ((long long)NT * UR) < nsr - 1
                                      ? nvec / ((long long)NT * UR) : (long long)(nsr - 1);
@@ -592,105 +782,123 @@ __global__ void __launch_bounds__(NT) k_resample(
     const long long extra[2] = {(chunk == 0 && (int)threadIdx.x < head) ? (long long)threadIdx.x : -1,
                                 (chunk == tail_chunk && tail < V && threadIdx.x < VEC) ? tail : -1};
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
+    for (int e = 0; e < 2; ++e)
       if (extra[e] >= 0)
         rs += res_weight(Dt<T>::load(pt + extra[e]), d.bonus ? 0.f : Dt<T>::load(pd + extra[e]), d);
-    }
   } else {  // rows of different alignment: scalar loads over the chunk
     const long long lo = chunk_lo(chunk), hi = chunk_hi(chunk);
     for (long long v = lo + threadIdx.x; v < hi; v += NT)
       rs += res_weight(Dt<T>::load(pt + v), d.bonus ? 0.f : Dt<T>::load(pd + v), d);
   }
 
-  // chunk sums (fp64 across threads)
-  __shared__ double sm_r[NWARP];
-  __shared__ int s_last;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const double r64 = warp_sum((double)rs);
-  if (lane == 0) sm_r[warp] = r64;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    double a = 0.0;
-    for (int w = 0; w < NWARP; ++w) a += sm_r[w];
-    ResPartial o;
-    o.R = a;
-    o.pad = 0.0;
-    rpart[b * nsr + chunk] = o;
-    __threadfence();
-    const unsigned t = atomicAdd(&counters[b], 1u);
-    s_last = (t == (unsigned)(nsr - 1));
+  // chunk sum (fp64 across threads) and the arrival ticket
+  {
+    double tot;
+    block_excl_scan((double)rs, tot);
+    if (threadIdx.x == 0) {
+      ResPartial o;
+      o.R = tot;
+      o.pad = 0.0;
+      rpart[b * nsr + chunk] = o;
+      __threadfence();
+      const unsigned t = atomicAdd(&counters[b], 1u);
+      s_last = (t == (unsigned)(nsr - 1));
+      s_chunk = INT_MAX;
+      s_y = INT_MAX;
+      s_lastpos = -1;
+    }
+    __syncthreads();
   }
-  __syncthreads();
   if (!s_last) return;
 
   // ---- the last CTA of sequence b draws ----
-  __shared__ double s_base, s_t;
-  __shared__ int s_chunk, s_mode, s_y, s_lastpos;
-  if (threadIdx.x == 0) {
-    __threadfence();
-    const ResPartial *rp = rpart + b * nsr;
-    double Z = 0.0;
-    for (int c2 = 0; c2 < nsr; ++c2) Z += __ldcg(&rp[c2].R);
-    s_y = INT_MAX;
-    s_lastpos = -1;
-    // Residual mass below 2^-64 (relative to the target row's largest
-    // probability): the fp32 weights have run out of range, so the draw is
-    // redone in fp64 over the whole row pair.
-    s_mode = (!d.bonus && !(Z >= ldexp(sl.St, -64))) ? 1 : 0;
-    if (s_mode == 0) {
-      const double t = (double)u_resample[b] * Z;
-      double acc = 0.0, base = -1.0;
-      int cs = -1;
-      for (int c2 = 0; c2 < nsr; ++c2) {
-        const double v = __ldcg(&rp[c2].R);
-        if (acc + v > t) {
-          cs = c2;
-          base = acc;
-          break;
-        }
-        acc += v;
+  __threadfence();
+  const ResPartial *rp = rpart + b * nsr;
+  const int cper = (nsr + NT - 1) / NT;  // chunks per thread, contiguous
+  const int c0 = threadIdx.x * cper < nsr ? threadIdx.x * cper : nsr;
+  const int c1 = c0 + cper < nsr ? c0 + cper : nsr;
+  double my = 0.0;
+  for (int c2 = c0; c2 < c1; ++c2) my += __ldcg(&rp[c2].R);
+  double Z;
+  const double cexcl = block_excl_scan(my, Z);
+  if (threadIdx.x == 0) s_mode = (!d.bonus && !(Z >= ldexp(St, -64))) ? 1 : 0;
+  __syncthreads();
+  if (s_mode == 1) {
+    const int y = draw_exact64(pt, pd, V, d.Mt, St, d.Md, Sd, c64, (double)ures, &s_y, &s_lastpos,
+                               dbg_Z ? dbg_Z + b : nullptr);
+    if (threadIdx.x == 0) out_tokens[b * (K + 1) + n] = y;
+    return;
+  }
+  const double t = (double)ures * Z;
+  {
+    double C = cexcl;
+    for (int c2 = c0; c2 < c1; ++c2) {
+      const double v = __ldcg(&rp[c2].R);
+      if (C <= t && t < C + v) {
+        atomicMin(&s_chunk, c2);
+        break;
       }
-      if (cs < 0) {  // defensive: rounding left t at or past the total
-        for (int c2 = nsr - 1; c2 >= 0 && cs < 0; --c2)
-          if (__ldcg(&rp[c2].R) > 0.0) cs = c2;
-        if (cs < 0) cs = 0;
-      }
-      s_base = base;  // < 0 selects the "last positive element" rule
-      s_t = t;
-      s_chunk = cs;
-      if (dbg_Z) dbg_Z[b] = Z / sl.St;
+      C += v;
     }
   }
   __syncthreads();
-  if (s_mode == 1) {
-    int y = draw_exact64(pt, pd, V, sl, (double)u_resample[b], &s_y, &s_lastpos,
-                         dbg_Z ? dbg_Z + b : nullptr);
-    if (threadIdx.x == 0) out_tokens[b * (K + 1) + sl.n] = y;
-    return;
+  if (threadIdx.x == 0) {
+    s_t = t;
+    s_base = -1.0;  // < 0 selects the "last positive element" rule
+    if (s_chunk == INT_MAX) {  // rounding left t at or past the total
+      int cs = 0;
+      for (int c2 = nsr - 1; c2 >= 0; --c2)
+        if (__ldcg(&rp[c2].R) > 0.0) {
+          cs = c2;
+          break;
+        }
+      s_chunk = cs;
+    }
+    if (dbg_Z) dbg_Z[b] = Z / St;
   }
+  __syncthreads();
+  // the owner of the chosen chunk publishes its exclusive prefix
+  if (s_chunk >= c0 && s_chunk < c1) {
+    double C = cexcl;
+    for (int c2 = c0; c2 < s_chunk; ++c2) C += __ldcg(&rp[c2].R);
+    const double v = __ldcg(&rp[s_chunk].R);
+    if (C <= t && t < C + v) s_base = C;
+  }
+  __syncthreads();
+
+  // rescan of the chosen chunk: contiguous elements per thread, in registers
   const long long lo = chunk_lo(s_chunk), hi = chunk_hi(s_chunk);
   const long long L = hi - lo;
-  const long long E = (L + NT - 1) / NT;  // contiguous elements per thread
+  const long long E = (L + NT - 1) / NT;
   const long long e0 = lo + (long long)threadIdx.x * E < hi ? lo + (long long)threadIdx.x * E : hi;
   const long long e1 = (e0 + E < hi) ? e0 + E : hi;
+  float w[EMAX];
+#pragma unroll
+  for (int k = 0; k < EMAX; ++k) {
+    const long long v = e0 + k;
+    w[k] = (v < e1) ? res_weight(Dt<T>::load(pt + v), d.bonus ? 0.f : Dt<T>::load(pd + v), d)
+                    : 0.0f;
+  }
   double mysum = 0.0;
   int lastpos = -1;
-  for (long long v = e0; v < e1; ++v) {
-    const float x = res_weight(Dt<T>::load(pt + v), d.bonus ? 0.f : Dt<T>::load(pd + v), d);
-    mysum += (double)x;
-    if (x > 0.0f) lastpos = (int)v;
+#pragma unroll
+  for (int k = 0; k < EMAX; ++k) {
+    mysum += (double)w[k];
+    if (w[k] > 0.0f) lastpos = (int)(e0 + k);
   }
-  double total;
-  const double excl = block_excl_scan(mysum, total);
+  double ctot;
+  const double excl = block_excl_scan(mysum, ctot);
   if (lastpos >= 0) atomicMax(&s_lastpos, lastpos);
   if (s_base >= 0.0) {
     double C = s_base + excl;
-    const double t = s_t;
-    for (long long v = e0; v < e1; ++v) {
-      C += (double)res_weight(Dt<T>::load(pt + v), d.bonus ? 0.f : Dt<T>::load(pd + v), d);
-      if (C > t) {
-        atomicMin(&s_y, (int)v);
-        break;
+#pragma unroll
+    for (int k = 0; k < EMAX; ++k) {
+      if (e0 + k < e1) {
+        C += (double)w[k];
+        if (C > t) {
+          atomicMin(&s_y, (int)(e0 + k));
+          break;
+        }
       }
     }
   }
@@ -698,15 +906,15 @@ __global__ void __launch_bounds__(NT) k_resample(
   if (threadIdx.x == 0) {
     int y = s_y;
     if (y == INT_MAX) y = (s_lastpos >= 0) ? s_lastpos : (int)lo;
-    out_tokens[b * (K + 1) + sl.n] = y;
+    out_tokens[b * (K + 1) + n] = y;
   }
 }
 
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-enum KernelId { KID_STATS = 0, KID_ACCEPT = 1, KID_RESAMPLE = 2, KID_COUNT = 3 };
-const char *kKernelNames[KID_COUNT] = {"k_row_stats", "k_accept", "k_resample"};
+enum KernelId { KID_STATS = 0, KID_FINISH = 1, KID_COUNT = 2 };
+const char *kKernelNames[KID_COUNT] = {"k_row_stats", "k_finish"};
 
 std::mutex g_mu;
 uint64_t g_launches[KID_COUNT];
@@ -726,9 +934,9 @@ std::unordered_map<int, DeviceBuf> g_staging;  // end-to-end staging per device
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct Plan {
-  int esize, vec, U, nsplit, UR, nsr;
-  long long rows;
-  size_t off_part, off_sel, off_rpart, off_cnt, total;
+  int esize, vec, U, tpr, slots, UR, nsr;
+  long long rows, tiles, G1;  // G1: CTAs of the statistics sweep
+  size_t off_part, off_rpart, off_cnt, total;
 };
 
 int num_sms() {
@@ -737,6 +945,10 @@ int num_sms() {
   return n > 0 ? n : 148;
 }
 
+constexpr int kStatsCtasPerSm = 4;  // 3-stage 16 KB rings: 4 CTAs fit an SM
+
+// Work decomposition for these sizes; a pure function of the sizes and the SM
+// count, so repeated calls reduce in the same order (bit-reproducible).
 bool make_plan(int B, int K, int V, specdec_dtype dtype, int sms, Plan &pl) {
   if (B < 0 || K < 1 || K > 32 || V < 1) return false;
   if (dtype != SPECDEC_F32 && dtype != SPECDEC_BF16) return false;
@@ -744,29 +956,78 @@ bool make_plan(int B, int K, int V, specdec_dtype dtype, int sms, Plan &pl) {
   pl.vec = 16 / pl.esize;
   pl.rows = (long long)B * (2 * K + 1);
   const long long nvec_max = ((long long)V + pl.vec - 1) / pl.vec;
-  // 4 vectors per thread when that still gives >= 4 CTAs per SM; otherwise 1,
-  // so that small batches (B = 1) still spread over every SM
-  const long long ns4 = (nvec_max + NT * 4 - 1) / (NT * 4);
-  pl.U = (pl.rows * ns4 >= 4LL * sms) ? 4 : 1;
-  const long long ns = (nvec_max + (long long)NT * pl.U - 1) / ((long long)NT * pl.U);
-  pl.nsplit = (int)(ns > 0 ? ns : 1);
+  // tiles of 4 vectors per consumer thread (16 KB); 1 vector per thread when
+  // 16 KB tiles would leave SMs idle (single-sequence batches)
+  const long long cap = (long long)kStatsCtasPerSm * sms;
+  long long tpr = (nvec_max + NTC * 4 - 1) / (NTC * 4);
+  pl.U = 4;
+  if (pl.rows * tpr < 2 * cap) {
+    pl.U = 1;
+    tpr = (nvec_max + NTC - 1) / NTC;
+  }
+  if (tpr < 1) tpr = 1;
+  pl.tpr = (int)tpr;
+  pl.tiles = pl.rows * tpr;
+  pl.G1 = pl.tiles < cap ? pl.tiles : cap;
+  // partial slots per row: the most CTAs whose tile ranges meet one row
+  const long long minr = pl.tiles / pl.G1;  // shortest range
+  pl.slots = (int)((tpr - 1 + minr - 1) / minr + 1);
   const long long nr2 = (nvec_max + NT * 2 - 1) / (NT * 2);
   pl.UR = ((long long)B * nr2 >= 2LL * sms) ? 2 : 1;
   const long long nr = (nvec_max + (long long)NT * pl.UR - 1) / ((long long)NT * pl.UR);
   pl.nsr = (int)(nr > 0 ? nr : 1);
-  if (pl.rows * pl.nsplit > INT_MAX || (long long)B * pl.nsr > INT_MAX) return false;
+  if ((long long)B * pl.nsr > INT_MAX) return false;
   if ((long long)B * (K + 1) * (long long)V > (1LL << 56)) return false;
   size_t off = 0;
   pl.off_part = off;
-  off = align256(off + sizeof(Partial) * (size_t)pl.rows * pl.nsplit);
-  pl.off_sel = off;
-  off = align256(off + sizeof(Sel) * (size_t)B);
+  off = align256(off + sizeof(Partial) * (size_t)pl.rows * pl.slots * CW);
   pl.off_rpart = off;
   off = align256(off + sizeof(ResPartial) * (size_t)B * pl.nsr);
   pl.off_cnt = off;
   off = align256(off + sizeof(unsigned) * (size_t)B);
   pl.total = off > 0 ? off : 256;
   return true;
+}
+
+// resident CTAs per SM of a kernel with the given block and dynamic shared
+// memory (queried once per device and kernel; also raises the kernel's
+// dynamic shared-memory limit to what it asks for)
+template <typename KernelT>
+int resident_ctas(KernelT kernel, int threads, size_t smem) {
+  static std::mutex mu;
+  static std::unordered_map<std::string, int> cache;  // (device, kernel) -> CTAs per SM
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const std::string key = std::to_string(dev) + ":" +
+                          std::to_string(reinterpret_cast<uintptr_t>((const void *)kernel));
+  std::lock_guard<std::mutex> lk(mu);
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem) != cudaSuccess ||
+      n < 1)
+    n = 1;
+  cache[key] = n;
+  return n;
+}
+
+// launch with programmatic stream serialisation: the kernel may be scheduled
+// while the previous one drains and waits for it with cudaGridDependencySynchronize
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, cudaStream_t st,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
 struct LaunchTimer {
@@ -799,35 +1060,37 @@ specdec_status launch_all(const void *tg, const void *dr, const int32_t *tok, co
   const T *t = static_cast<const T *>(tg);
   const T *d = static_cast<const T *>(dr);
   Partial *part = reinterpret_cast<Partial *>(ws + pl.off_part);
-  Sel *sel = reinterpret_cast<Sel *>(ws + pl.off_sel);
   ResPartial *rp = reinterpret_cast<ResPartial *>(ws + pl.off_rpart);
   unsigned *cnt = reinterpret_cast<unsigned *>(ws + pl.off_cnt);
-  const unsigned g1 = (unsigned)(pl.rows * pl.nsplit);
+  StatsGeom g;
+  g.K = K;
+  g.V = V;
+  g.tpr = pl.tpr;
+  g.tiles = pl.tiles;
+  g.slots = pl.slots;
+  cudaError_t e = cudaSuccess;
   {
     LaunchTimer lt(KID_STATS, st);
-    if (pl.U == 4)
-      k_row_stats<T, 4><<<g1, NT, 0, st>>>(t, d, temp, K, V, pl.nsplit, part);
-    else
-      k_row_stats<T, 1><<<g1, NT, 0, st>>>(t, d, temp, K, V, pl.nsplit, part);
+    auto kern = pl.U == 4 ? k_row_stats<T, 4> : k_row_stats<T, 1>;
+    const size_t smem = (size_t)NSTAGE * NTC * pl.U * 16;
+    // the sweep assumes its CTAs are co-resident only for speed, not for
+    // progress: nothing waits on another CTA
+    resident_ctas(kern, NTS, smem);
+    kern<<<(unsigned)pl.G1, NTS, smem, st>>>(t, d, temp, g, part, cnt, B);
+    e = cudaGetLastError();
   }
+  if (e != cudaSuccess) return SPECDEC_ECUDA;
   {
-    LaunchTimer lt(KID_ACCEPT, st);
-    k_accept<T><<<(unsigned)((B + 3) / 4), 128, 0, st>>>(
-        t, d, tok, ua, temp, B, K, V, pl.nsplit, part, sel, cnt, out_tokens, out_n,
-        dbg ? dbg->row_max : nullptr, dbg ? dbg->row_sum : nullptr, dbg ? dbg->p_x : nullptr,
-        dbg ? dbg->q_x : nullptr);
+    LaunchTimer lt(KID_FINISH, st);
+    const unsigned g2 = (unsigned)((long long)B * pl.nsr);
+    auto kern = pl.UR == 2 ? k_finish<T, 2> : k_finish<T, 1>;
+    e = launch_pdl(kern, g2, NT, st, t, d, tok, ua, ur, temp, K, (long long)V, pl.tpr, pl.tiles,
+                   pl.G1, pl.slots, pl.nsr,
+                   (const Partial *)part, rp, cnt, out_tokens, out_n,
+                   dbg ? dbg->row_max : nullptr, dbg ? dbg->row_sum : nullptr,
+                   dbg ? dbg->p_x : nullptr, dbg ? dbg->q_x : nullptr, dbg ? dbg->Z : nullptr);
   }
-  {
-    LaunchTimer lt(KID_RESAMPLE, st);
-    const unsigned g3 = (unsigned)((long long)B * pl.nsr);
-    if (pl.UR == 2)
-      k_resample<T, 2><<<g3, NT, 0, st>>>(t, d, ur, K, V, pl.nsr, sel, rp, cnt, out_tokens,
-                                          dbg ? dbg->Z : nullptr);
-    else
-      k_resample<T, 1><<<g3, NT, 0, st>>>(t, d, ur, K, V, pl.nsr, sel, rp, cnt, out_tokens,
-                                          dbg ? dbg->Z : nullptr);
-  }
-  return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ECUDA;
+  return e == cudaSuccess ? SPECDEC_OK : SPECDEC_ECUDA;
 }
 
 specdec_status check_args(const void *tg, const void *dr, const int32_t *tok, const float *ua,
