@@ -224,6 +224,7 @@ def cpu_baseline(x, w, seconds):
 def run_cuda(args):
     import torch
     import speculative_sampling_b200 as sd
+    from speculative_sampling_b200 import dist as sdist
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -241,8 +242,7 @@ def run_cuda(args):
     dev = torch.device("cuda", local)
     w = inputs.WORKLOADS[args.workload]
     # weak scaling: rank r verifies sequences [r*B, (r+1)*B)
-    x = inputs.generate(args.workload, seq_begin=rank * w.B, seq_end=(rank + 1) * w.B,
-                        B=w.B * world)
+    x = sdist.generate_shard(args.workload, rank, world)
     B, K, V = x.B, x.K, x.V
     dt_code = sd.SPECDEC_BF16 if w.dtype == "bf16" else sd.SPECDEC_F32
     floor = x.floor_bytes
@@ -305,7 +305,7 @@ def run_cuda(args):
     sampler.window = (tw0, tw1)
     sampler.stop()
     after = [L.specdec_launch_count(i) for i in range(nk)]
-    ms = e0.elapsed_time(e1)
+    ms = sdist.max_over_ranks(e0.elapsed_time(e1), dev)
     # kernel region: the same K steps again with every launch bracketed by CUDA
     # events on its stream; gives each kernel's mean device time (roofline)
     kern = {}
@@ -315,10 +315,6 @@ def run_cuda(args):
             step(i)
         torch.cuda.synchronize()
         kern = sd.profile_end()
-    if dist is not None:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
     ms_step = ms / args.steps
     total_bytes = floor * world
     gbs = total_bytes / (ms_step * 1e-3) / 1e9
@@ -345,12 +341,8 @@ def run_cuda(args):
         L.specdec_verify_host(*hargs)
     ee1.record(stream)
     torch.cuda.synchronize()
-    ms_e2e = ee0.elapsed_time(ee1)
-    if dist is not None:
-        t = torch.tensor([ms_e2e], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
-        barrier()
+    ms_e2e = sdist.max_over_ranks(ee0.elapsed_time(ee1), dev)
+    barrier()
     if not np.array_equal(hot.numpy(), ref_tok.numpy()):
         raise RuntimeError("end-to-end outputs differ from the device-resident run")
     e2e_gbs = total_bytes / (ms_e2e / args.e2e_steps * 1e-3) / 1e9

@@ -37,6 +37,7 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <cfloat>
 #include <climits>
 #include <cstring>
 #include <mutex>
@@ -146,17 +147,6 @@ __device__ __forceinline__ int row_head(const T *p, long long V) {
   return (int)(h < V ? h : V);
 }
 
-// Online update of (m, s) = (running max, sum 2^((z-m)c)) with one logit.
-// NaN propagates into s; +Inf makes m = +Inf (the row is rejected later).
-__device__ __forceinline__ void online_add(float &m, float &s, float x, Scale c) {
-  if (!(x <= m)) {
-    s = s * ex2(scaled(m - x, c)) + 1.0f;
-    m = x;
-  } else if (m != -INFINITY) {
-    s += ex2(scaled(x - m, c));
-  }
-}
-
 __device__ __forceinline__ double warp_sum(double v) {
 #pragma unroll
   for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
@@ -194,6 +184,9 @@ constexpr int NTC = CW * 32;        // consumer threads
 constexpr int NTS = NTC + 32;       // + one producer warp
 constexpr int NSTAGE = 3;           // depth of the shared-memory ring
 constexpr unsigned kWaitLimit = 1u << 22;  // try_wait rounds before giving up
+constexpr int kStatsCtasPerSm = 4;  // resident CTAs per SM the sweep is sized for
+constexpr int kFinishUW = 4;        // vectors per lane in a k_finish chunk
+constexpr int kFinishCtasPerSm = 4; // k_finish grids fit one wave of this many CTAs per SM
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -235,13 +228,6 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, unsigned b
       ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
-__device__ __forceinline__ uint4 lds128(const void *p) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(smem_u32(p)));
-  return v;
-}
 // pairs (x0, x1) of the 8 (bf16) or 4 (fp32) values of a 16-byte vector
 template <typename T>
 struct Pairs;
@@ -262,43 +248,88 @@ struct Pairs<float> {
   }
 };
 
-// Fold one 16-byte vector into the thread's (m, s): the vector's max by a
-// depth-3 FMNMX tree (NaN propagating), a rescale of s when the running max
-// grows, then packed fp32x2 exponent arguments, MUFU ex2 and a pairwise
-// packed sum.  Only the vector's 8 (bf16) or 4 (fp32) values are live.
+__device__ __forceinline__ float fmax3_nan(float a, float b, float c) {
+  float y;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
+  return y;
+}
+
+// Per-thread statistics of a row segment, kept against a lazy reference:
+//   r    the exponent reference: acc.x + acc.y = sum 2^((z - r) c) so far;
+//   mt   the true running max.
+// r moves only when the running max passes it by more than thr = 64/c (a
+// term would pass 2^64); with logits this happens once at the start of a row
+// and almost never again, so warps do not diverge on running-max updates.
+// Terms stay below 2^64 (far inside fp32), and fp32 precision is scale free,
+// so nothing is lost.  At the end of the segment the sum is moved to the true
+// max once.  The sum is kept as a packed fp32 pair (one FADD2 per vector).
+struct RunStat {
+  float r, mt;
+  float2 acc;
+};
+__device__ __forceinline__ void runstat_init(RunStat &q) {
+  q.r = -INFINITY;
+  q.mt = -INFINITY;
+  q.acc = make_float2(0.0f, 0.0f);
+}
+// rare path: the running max passed the reference (also the first finite value)
+__device__ __forceinline__ void runstat_rebase(RunStat &q, Scale c) {
+  if (q.r != -INFINITY) {
+    const float f = ex2(scaled(q.r - q.mt, c));
+    q.acc = __fmul2_rn(q.acc, make_float2(f, f));
+  }
+  q.r = q.mt;
+}
+// sum expressed against the true max (call once, at the end of a segment)
+__device__ __forceinline__ float runstat_sum_at_max(const RunStat &q, Scale c) {
+  const float s = q.acc.x + q.acc.y;
+  if (q.r == q.mt || !(q.r > -INFINITY) || !isfinite(q.mt)) return s;
+  return s * ex2(scaled(q.r - q.mt, c));
+}
+
+// Fold one 16-byte vector: the running max with three-input NaN-propagating
+// FMNMX, then packed fp32x2 exponent arguments against r, MUFU ex2 and a
+// pairwise packed sum.  Only the vector's 8 (bf16) or 4 (fp32) values are live.
 template <typename T>
-__device__ __forceinline__ void vec_fold(const uint4 &v, float &m, float &s, Scale c) {
+__device__ __forceinline__ void vec_fold(const uint4 &v, RunStat &q, Scale c, float thr) {
   constexpr int N = Pairs<T>::N;
   float2 x[N];
 #pragma unroll
-  for (int q = 0; q < N; ++q) x[q] = Pairs<T>::get(v, q);
-  float mx[N];
+  for (int k = 0; k < N; ++k) x[k] = Pairs<T>::get(v, k);
+  if (N == 4) {
+    const float a = fmax3_nan(x[0].x, x[0].y, x[1].x);
+    const float b = fmax3_nan(x[1].y, x[2].x, x[2].y);
+    const float d = fmax3_nan(x[N - 1].x, x[N - 1].y, q.mt);
+    q.mt = fmax3_nan(a, b, d);
+  } else {
+    q.mt = fmax3_nan(fmax3_nan(x[0].x, x[0].y, x[N - 1].x), x[N - 1].y, q.mt);
+  }
+  if (q.mt > q.r + thr) runstat_rebase(q, c);
+  // while every value so far is -inf (r = -inf) the reference is clamped to
+  // -FLT_MAX so the -inf values give exactly 0 instead of NaN
+  const float rr = fmaxf(q.r, -FLT_MAX);
+  const float2 nr = make_float2(-rr, -rr), hi = make_float2(c.hi, c.hi),
+               lo = make_float2(c.lo, c.lo);
+  float2 e[N];
 #pragma unroll
-  for (int q = 0; q < N; ++q) mx[q] = fmax_nan(x[q].x, x[q].y);
+  for (int k = 0; k < N; ++k) {
+    const float2 d = __fadd2_rn(x[k], nr);
+    const float2 a = __ffma2_rn(d, hi, __fmul2_rn(d, lo));
+    e[k] = make_float2(ex2(a.x), ex2(a.y));
+  }
 #pragma unroll
   for (int w = 1; w < N; w *= 2)
 #pragma unroll
-    for (int q = 0; q + w < N; q += 2 * w) mx[q] = fmax_nan(mx[q], mx[q + w]);
-  if (!(mx[0] <= m)) {  // new running max (or NaN): rescale what we have
-    s = s * ex2(scaled(m - mx[0], c));
-    m = mx[0];
-  }
-  if (m != -INFINITY) {
-    const float2 nm = make_float2(-m, -m), hi = make_float2(c.hi, c.hi),
-                 lo = make_float2(c.lo, c.lo);
-    float2 e[N];
-#pragma unroll
-    for (int q = 0; q < N; ++q) {
-      const float2 d = __fadd2_rn(x[q], nm);
-      const float2 a = __ffma2_rn(d, hi, __fmul2_rn(d, lo));
-      e[q] = make_float2(ex2(a.x), ex2(a.y));
-    }
-#pragma unroll
-    for (int w = 1; w < N; w *= 2)
-#pragma unroll
-      for (int q = 0; q + w < N; q += 2 * w) e[q] = __fadd2_rn(e[q], e[q + w]);
-    s += e[0].x + e[0].y;
-  }
+    for (int k = 0; k + w < N; k += 2 * w) e[k] = __fadd2_rn(e[k], e[k + w]);
+  q.acc = __fadd2_rn(q.acc, e[0]);
+}
+
+// the same for one scalar logit (row heads and tails)
+__device__ __forceinline__ void elem_fold(float x, RunStat &q, Scale c, float thr) {
+  q.mt = fmax_nan(q.mt, x);
+  if (q.mt > q.r + thr) runstat_rebase(q, c);
+  const float rr = fmaxf(q.r, -FLT_MAX);
+  q.acc.x += ex2(scaled(x - rr, c));
 }
 
 struct StatsGeom {
@@ -358,7 +389,7 @@ struct RowCursor {
 };
 
 template <typename T, int U>
-__global__ void __launch_bounds__(NTS) k_row_stats(const T *__restrict__ target,
+__global__ void __launch_bounds__(NTS, kStatsCtasPerSm) k_row_stats(const T *__restrict__ target,
                                                    const T *__restrict__ draft,
                                                    const float *__restrict__ temperature,
                                                    StatsGeom g, Partial *__restrict__ part,
@@ -388,27 +419,40 @@ __global__ void __launch_bounds__(NTS) k_row_stats(const T *__restrict__ target,
   __syncthreads();
   if (t0 >= t1) return;
 
+  // The CTA's tiles [t0, t1) are walked as row segments: the tiles of one row
+  // that fall in the range.  Inside a segment the full tiles come first (no
+  // per-element predicates), then at most one partial tile.
+  const long long row_first = t0 / g.tpr, row_last = (t1 - 1) / g.tpr;
+
   if (warp == CW) {  // ---------------- producer warp ----------------
     if (lane != 0) return;
-    unsigned it = 0;
+    unsigned it = 0, ph = 0;  // copies issued; phase parity of the current ring pass
+    int st = 0;               // ring slot of the next copy
     RowCursor<T> rc;
     rc.start(target, draft, g, t0);
-    for (long long t = t0; t < t1 && !*(volatile int *)&s_abort; ++t) {
-      if (rc.ti == g.tpr) rc.next_row(target, draft, g);
-      const long long v0 = (long long)rc.ti * TV;
-      const long long v1 = (v0 + TV < rc.nvec) ? v0 + TV : rc.nvec;
-      ++rc.ti;
-      if (v0 >= v1) continue;  // an empty last tile (the row's tail is scalar)
-      const int st = (int)(it % NSTAGE);
-      if (!mbar_wait(&empty[st], ((it / NSTAGE) & 1u) ^ 1u)) {
-        atomicExch(&s_abort, 1);
-        break;
+    for (long long row = row_first; row <= row_last; ++row) {
+      if (row != row_first) rc.next_row(target, draft, g);
+      const int tb = (row == row_first) ? (int)(t0 - row * g.tpr) : 0;
+      const int te = (row == row_last) ? (int)(t1 - row * g.tpr) : g.tpr;
+      for (int ti = tb; ti < te; ++ti) {
+        const long long v0 = (long long)ti * TV;
+        const long long v1 = (v0 + TV < rc.nvec) ? v0 + TV : rc.nvec;
+        if (v0 >= v1) break;  // the rest of the row is its scalar tail
+        if (*(volatile int *)&s_abort || !mbar_wait(&empty[st], ph ^ 1u)) {
+          atomicExch(&s_abort, 1);
+          goto drain;
+        }
+        const unsigned bytes = (unsigned)(v1 - v0) * 16u;
+        mbar_arrive_tx(&full[st], bytes);
+        bulk_load(ring + (size_t)st * TILE_BYTES, rc.pv + v0, bytes, &full[st]);
+        ++it;
+        if (++st == NSTAGE) {
+          st = 0;
+          ph ^= 1u;
+        }
       }
-      const unsigned bytes = (unsigned)(v1 - v0) * 16u;
-      mbar_arrive_tx(&full[st], bytes);
-      bulk_load(ring + (size_t)st * TILE_BYTES, rc.pv + v0, bytes, &full[st]);
-      ++it;
     }
+  drain:
     // The CTA must not retire with copies in flight: wait (bounded) until the
     // last copy issued into each slot has landed.
     for (unsigned k = 0; k < NSTAGE && k < it; ++k) {
@@ -420,75 +464,102 @@ __global__ void __launch_bounds__(NTS) k_row_stats(const T *__restrict__ target,
 
   // ---------------- consumer warps ----------------
   // No CTA-wide barrier inside the walk: each warp folds its share of every
-  // tile and, at the end of a row (or of the CTA's range), reduces its lanes
-  // and writes its own partial.  After an abort the waits and the arithmetic
-  // are skipped.
-  unsigned it = 0;
+  // tile and, at the end of a row segment, reduces its lanes and writes its own
+  // partial.  After an abort the waits and the arithmetic are skipped (every
+  // warp still walks the same tiles).
+  unsigned ph = 0;  // phase parity of the current ring pass
+  int st = 0;       // ring slot of the next tile
   RowCursor<T> rc;
   rc.start(target, draft, g, t0);
   Scale c = make_scale(kLog2e / (double)__ldg(temperature + rc.b));
+  float thr = 64.0f / c.hi;
   // temperature of the sequence after this one, fetched a row ahead
   float T_next = (rc.b + 1 < B) ? __ldg(temperature + rc.b + 1) : 1.0f;
-  float m = -INFINITY, s = 0.0f;
-  int seg_first = rc.ti;  // first tile of this row in this CTA's range
-  for (long long t = t0; t < t1; ++t) {
-    const long long v0 = (long long)rc.ti * TV;
-    const long long v1 = (v0 + TV < rc.nvec) ? v0 + TV : rc.nvec;
-    if (v0 < v1) {
-      const int st = (int)(it % NSTAGE);
+  for (long long row = row_first; row <= row_last; ++row) {
+    if (row != row_first) {
+      const bool new_seq = (rc.j == 2 * g.K);
+      rc.next_row(target, draft, g);
+      if (new_seq) {
+        c = make_scale(kLog2e / (double)T_next);
+        thr = 64.0f / c.hi;
+        T_next = (rc.b + 1 < B) ? __ldg(temperature + rc.b + 1) : 1.0f;
+      }
+    }
+    const int tb = (row == row_first) ? (int)(t0 - row * g.tpr) : 0;
+    const int te = (row == row_last) ? (int)(t1 - row * g.tpr) : g.tpr;
+    const long long full_tiles = rc.nvec / TV;  // tiles with all TV vectors
+    const int tf = (int)((long long)te < full_tiles ? te : full_tiles);
+    RunStat q;
+    runstat_init(q);
+    // full tiles
+    for (int ti = tb; ti < tf; ++ti) {
       bool have = false;
       if (!*(volatile int *)&s_abort) {
-        have = __all_sync(FULL, mbar_wait(&full[st], (it / NSTAGE) & 1u));
+        have = __all_sync(FULL, mbar_wait(&full[st], ph));
         if (!have && lane == 0) atomicExch(&s_abort, 1);
       }
-      ++it;
+      const uint4 *tile = reinterpret_cast<const uint4 *>(ring + (size_t)st * TILE_BYTES);
+      if (++st == NSTAGE) {
+        st = 0;
+        ph ^= 1u;
+      }
+      if (!have) continue;
+      uint4 v[U];
+#pragma unroll
+      for (int k = 0; k < U; ++k) v[k] = tile[k * NTC + threadIdx.x];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st == 0 ? NSTAGE - 1 : st - 1]);
+#pragma unroll
+      for (int k = 0; k < U; ++k) vec_fold<T>(v[k], q, c, thr);
+    }
+    // at most one partial tile (the row's last vectors)
+    const int tpb = tb > tf ? tb : tf;
+    if (tpb < te && (long long)tpb * TV < rc.nvec) {
+      const long long nv = rc.nvec - (long long)tpb * TV;
+      bool have = false;
+      if (!*(volatile int *)&s_abort) {
+        have = __all_sync(FULL, mbar_wait(&full[st], ph));
+        if (!have && lane == 0) atomicExch(&s_abort, 1);
+      }
+      const uint4 *tile = reinterpret_cast<const uint4 *>(ring + (size_t)st * TILE_BYTES);
+      const int cur = st;
+      if (++st == NSTAGE) {
+        st = 0;
+        ph ^= 1u;
+      }
       if (have) {
-        const long long nv = v1 - v0;
-        const unsigned char *tile = ring + (size_t)st * TILE_BYTES;
         uint4 v[U];
 #pragma unroll
         for (int k = 0; k < U; ++k) {
           const int vi = k * NTC + threadIdx.x;
-          v[k] = (vi < nv) ? lds128(tile + (size_t)vi * 16) : Dt<T>::neg_inf();
+          v[k] = (vi < nv) ? tile[vi] : Dt<T>::neg_inf();
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[st]);
+        if (lane == 0) mbar_arrive(&empty[cur]);
 #pragma unroll
-        for (int k = 0; k < U; ++k) vec_fold<T>(v[k], m, s, c);
+        for (int k = 0; k < U; ++k) vec_fold<T>(v[k], q, c, thr);
       }
     }
-    ++rc.ti;
-    if (rc.ti == g.tpr || t + 1 == t1) {  // end of this CTA's part of the row
-      // scalar head / tail of the row when this CTA holds its first / last tile
-      if (seg_first == 0 && (int)threadIdx.x < rc.head)
-        online_add(m, s, Dt<T>::load(rc.p + threadIdx.x), c);
-      if (rc.ti == g.tpr) {
-        const long long tt = rc.head + rc.nvec * VEC + threadIdx.x;
-        if (tt < g.V) online_add(m, s, Dt<T>::load(rc.p + tt), c);
-      }
-      // this warp's partial: lanes combined in fp64 with shuffles
-      const float mw = warp_max_nan(m);
-      double sw = (m == -INFINITY) ? 0.0 : (double)s * (double)ex2(scaled(m - mw, c));
-      sw = warp_sum(sw);
-      if (lane == 0) {
-        const long long slot = (long long)blockIdx.x - tile_owner(rc.row * g.tpr, G, g.tiles);
-        Partial out;
-        out.s = sw;
-        out.m = mw;
-        out.pad = 0;
-        part[(rc.row * g.slots + slot) * CW + warp] = out;
-      }
-      if (t + 1 < t1) {  // next row
-        const bool new_seq = (rc.j == 2 * g.K);
-        rc.next_row(target, draft, g);
-        if (new_seq) {
-          c = make_scale(kLog2e / (double)T_next);
-          T_next = (rc.b + 1 < B) ? __ldg(temperature + rc.b + 1) : 1.0f;
-        }
-        m = -INFINITY;
-        s = 0.0f;
-        seg_first = 0;
-      }
+    // scalar head / tail of the row when this CTA holds its first / last tile
+    if (tb == 0 && (int)threadIdx.x < rc.head)
+      elem_fold(Dt<T>::load(rc.p + threadIdx.x), q, c, thr);
+    if (te == g.tpr) {
+      const long long tt = rc.head + rc.nvec * VEC + threadIdx.x;
+      if (tt < g.V) elem_fold(Dt<T>::load(rc.p + tt), q, c, thr);
+    }
+    // this warp's partial: lanes combined in fp64 with shuffles
+    const float m = q.mt;
+    const float sl = runstat_sum_at_max(q, c);
+    const float mw = warp_max_nan(m);
+    double sw = (m == -INFINITY) ? 0.0 : (double)sl * (double)ex2(scaled(m - mw, c));
+    sw = warp_sum(sw);
+    if (lane == 0) {
+      const long long slot = (long long)blockIdx.x - tile_owner(row * g.tpr, G, g.tiles);
+      Partial out;
+      out.s = sw;
+      out.m = mw;
+      out.pad = 0;
+      part[(row * g.slots + slot) * CW + warp] = out;
     }
   }
 }
@@ -604,27 +675,29 @@ __device__ __noinline__ int draw_exact64(const T *pt, const T *pd, long long V, 
   return y;
 }
 
-template <typename T, int UR>
-__global__ void __launch_bounds__(NT) k_finish(
+template <typename T, int UW>
+__global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
     const T *__restrict__ target, const T *__restrict__ draft,
     const int32_t *__restrict__ tokens, const float *__restrict__ u_accept,
     const float *__restrict__ u_resample, const float *__restrict__ temperature, int K,
-    long long V, int tpr, long long tiles, long long G1, int slots, int nsr,
+    long long V, int tpr, long long tiles, long long G1, int slots, int nsr, int cpb,
     const Partial *__restrict__ part,
     ResPartial *__restrict__ rpart, unsigned *__restrict__ counters,
     int32_t *__restrict__ out_tokens, int32_t *__restrict__ out_n,
     float *__restrict__ dbg_row_max, double *__restrict__ dbg_row_sum,
     double *__restrict__ dbg_px, double *__restrict__ dbg_qx, double *__restrict__ dbg_Z) {
   constexpr int VEC = Dt<T>::VEC;
-  constexpr long long CH = (long long)NT * UR * VEC;  // elements per chunk
-  constexpr int EMAX = UR * VEC + 1;                  // rescan elements per thread
+  constexpr long long CHV = 32LL * UW;                 // vectors per (warp-)chunk
+  constexpr long long CH = CHV * VEC;                  // elements per chunk
+  constexpr int EMAX = (int)((CH + 2 * VEC + NT - 1) / NT);  // rescan elements per thread
   __shared__ float sM[65];
   __shared__ double sS[65];
   __shared__ int s_n, s_last, s_mode, s_chunk, s_y, s_lastpos;
   __shared__ double s_base, s_t;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const long long b = (long long)blockIdx.x / nsr;
-  const int chunk = (int)((long long)blockIdx.x - b * nsr);
+  const int ncb = (nsr + cpb - 1) / cpb;  // CTAs per sequence
+  const long long b = (long long)blockIdx.x / ncb;
+  const int cb = (int)((long long)blockIdx.x - b * ncb);  // this CTA: chunks cb*cpb ...
   const int R = 2 * K + 1;
 
   // ---- inputs of this call (independent of the statistics kernel) ----
@@ -654,11 +727,18 @@ __global__ void __launch_bounds__(NT) k_finish(
     // row, in order, CW consumer warps each
     const int nslot = (int)(tile_owner(row * tpr + tpr - 1, G1, tiles) -
                             tile_owner(row * tpr, G1, tiles) + 1) * CW;
-    float m = -INFINITY;
-    for (int s = lane; s < nslot; s += 32) m = fmaxf(m, P[s].m);
+    // first 32 partials in registers (one load per lane), the rest streamed
+    Partial p0;
+    p0.m = -INFINITY;
+    p0.s = 0.0;
+    if (lane < nslot) p0 = P[lane];
+    float m = p0.m;
+    for (int s = lane + 32; s < nslot; s += 32) m = fmaxf(m, P[s].m);
     m = warp_max_nan(m);
-    double acc = 0.0;
-    for (int s = lane; s < nslot; s += 32) {
+    double acc = (lane < nslot)
+                     ? ((p0.m == -INFINITY) ? p0.s : p0.s * exp2(((double)p0.m - (double)m) * c64))
+                     : 0.0;
+    for (int s = lane + 32; s < nslot; s += 32) {
       const Partial ps = P[s];
       acc += (ps.m == -INFINITY) ? ps.s : ps.s * exp2(((double)ps.m - (double)m) * c64);
     }
@@ -666,8 +746,8 @@ __global__ void __launch_bounds__(NT) k_finish(
     if (lane == 0) {
       sM[r] = m;
       sS[r] = acc;
-      if (chunk == 0 && dbg_row_max) dbg_row_max[b * R + r] = m;
-      if (chunk == 0 && dbg_row_sum) dbg_row_sum[b * R + r] = acc;
+      if (cb == 0 && dbg_row_max) dbg_row_max[b * R + r] = m;
+      if (cb == 0 && dbg_row_sum) dbg_row_sum[b * R + r] = acc;
     }
   }
   __syncthreads();
@@ -695,7 +775,7 @@ __global__ void __launch_bounds__(NT) k_finish(
     const unsigned rej = ~accm & kmask;
     const int n = seq_ok ? (rej ? __ffs(rej) - 1 : K) : -1;
     if (lane == 0) s_n = n;
-    if (chunk == 0) {
+    if (cb == 0) {
       int32_t *ot = out_tokens + b * (K + 1);
       if (!seq_ok) {
         for (int i = lane; i <= K; i += 32) ot[i] = -1;
@@ -753,62 +833,69 @@ __global__ void __launch_bounds__(NT) k_finish(
     return v < V ? v : V;
   };
 
-  float rs = 0.f;
-  if (vec_ok) {
-    const uint4 *vt = reinterpret_cast<const uint4 *>(pt + head);
-    const uint4 *vd = reinterpret_cast<const uint4 *>(pd + head);
-    uint4 at[UR], ad[UR];
+  // Chunk sums: the warps of this CTA take its chunks round robin; a chunk is
+  // 32 lanes x UW vectors of the row pair, summed per lane in fp32 and across
+  // the warp in fp64 with shuffles (no CTA barrier).  Then one arrival ticket.
+  const uint4 *vt = reinterpret_cast<const uint4 *>(pt + head);
+  const uint4 *vd = reinterpret_cast<const uint4 *>(pd + head);
+  const long long tail_chunk = nvec / CHV < nsr - 1 ? nvec / CHV : (long long)(nsr - 1);
+  const int c_beg = cb * cpb;
+  const int c_end = (cb + 1) * cpb < nsr ? (cb + 1) * cpb : nsr;
+  bool wrote = false;
+  for (int chunk = c_beg + warp; chunk < c_end; chunk += NWARP) {
+    float rs = 0.f;
+    if (vec_ok) {
+      uint4 at[UW], ad[UW];
 #pragma unroll
-    for (int k = 0; k < UR; ++k) {
-      const long long vi = (long long)chunk * NT * UR + (long long)k * NT + threadIdx.x;
-      at[k] = vi < nvec ? __ldg(vt + vi) : make_uint4(0, 0, 0, 0);
-      ad[k] = (vi < nvec && !d.bonus) ? __ldg(vd + vi) : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int k = 0; k < UR; ++k) {
-      const long long vi = (long long)chunk * NT * UR + (long long)k * NT + threadIdx.x;
-      if (vi < nvec) {
-        float xt[VEC], xd[VEC];
-        Dt<T>::unpack(at[k], xt);
-        Dt<T>::unpack(ad[k], xd);
-#pragma unroll
-        for (int q = 0; q < VEC; ++q) rs += res_weight(xt[q], xd[q], d);
+      for (int k = 0; k < UW; ++k) {
+        const long long vi = (long long)chunk * CHV + (long long)k * 32 + lane;
+        at[k] = vi < nvec ? __ldg(vt + vi) : make_uint4(0, 0, 0, 0);
+        ad[k] = (vi < nvec && !d.bonus) ? __ldg(vd + vi) : make_uint4(0, 0, 0, 0);
       }
-    }
-    // (a thread may own one head and one tail element of the same chunk)
-    const long long tail_chunk = nvec / ((long long)NT * UR) < nsr - 1
-                                     ? nvec / ((long long)NT * UR) : (long long)(nsr - 1);
-    const long long tail = head + nvec * VEC + threadIdx.x;
-    const long long extra[2] = {(chunk == 0 && (int)threadIdx.x < head) ? (long long)threadIdx.x : -1,
-                                (chunk == tail_chunk && tail < V && threadIdx.x < VEC) ? tail : -1};
 #pragma unroll
-    for (int e = 0; e < 2; ++e)
-      if (extra[e] >= 0)
-        rs += res_weight(Dt<T>::load(pt + extra[e]), d.bonus ? 0.f : Dt<T>::load(pd + extra[e]), d);
-  } else {  // rows of different alignment: scalar loads over the chunk
-    const long long lo = chunk_lo(chunk), hi = chunk_hi(chunk);
-    for (long long v = lo + threadIdx.x; v < hi; v += NT)
-      rs += res_weight(Dt<T>::load(pt + v), d.bonus ? 0.f : Dt<T>::load(pd + v), d);
-  }
-
-  // chunk sum (fp64 across threads) and the arrival ticket
-  {
-    double tot;
-    block_excl_scan((double)rs, tot);
-    if (threadIdx.x == 0) {
+      for (int k = 0; k < UW; ++k) {
+        const long long vi = (long long)chunk * CHV + (long long)k * 32 + lane;
+        if (vi < nvec) {
+          float xt[VEC], xd[VEC];
+          Dt<T>::unpack(at[k], xt);
+          Dt<T>::unpack(ad[k], xd);
+#pragma unroll
+          for (int q = 0; q < VEC; ++q) rs += res_weight(xt[q], xd[q], d);
+        }
+      }
+      // head elements (chunk 0) and the < VEC tail elements (their chunk)
+      const long long tail = head + nvec * VEC + lane;
+      const long long extra[2] = {(chunk == 0 && lane < head) ? (long long)lane : -1,
+                                  (chunk == tail_chunk && tail < V && lane < VEC) ? tail : -1};
+#pragma unroll
+      for (int e = 0; e < 2; ++e)
+        if (extra[e] >= 0)
+          rs += res_weight(Dt<T>::load(pt + extra[e]), d.bonus ? 0.f : Dt<T>::load(pd + extra[e]),
+                           d);
+    } else {  // rows of different alignment: scalar loads over the chunk
+      const long long lo = chunk_lo(chunk), hi = chunk_hi(chunk);
+      for (long long v = lo + lane; v < hi; v += 32)
+        rs += res_weight(Dt<T>::load(pt + v), d.bonus ? 0.f : Dt<T>::load(pd + v), d);
+    }
+    const double tot = warp_sum((double)rs);
+    if (lane == 0) {
       ResPartial o;
       o.R = tot;
       o.pad = 0.0;
       rpart[b * nsr + chunk] = o;
-      __threadfence();
-      const unsigned t = atomicAdd(&counters[b], 1u);
-      s_last = (t == (unsigned)(nsr - 1));
-      s_chunk = INT_MAX;
-      s_y = INT_MAX;
-      s_lastpos = -1;
+      wrote = true;
     }
-    __syncthreads();
   }
+  if (wrote) __threadfence();  // chunk sums visible before this CTA's ticket
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const unsigned t = atomicAdd(&counters[b], 1u);
+    s_last = (t == (unsigned)(ncb - 1));
+    s_chunk = INT_MAX;
+    s_y = INT_MAX;
+    s_lastpos = -1;
+  }
+  __syncthreads();
   if (!s_last) return;
 
   // ---- the last CTA of sequence b draws ----
@@ -934,7 +1021,7 @@ std::unordered_map<int, DeviceBuf> g_staging;  // end-to-end staging per device
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct Plan {
-  int esize, vec, U, tpr, slots, UR, nsr;
+  int esize, vec, U, tpr, slots, nsr, cpb;
   long long rows, tiles, G1;  // G1: CTAs of the statistics sweep
   size_t off_part, off_rpart, off_cnt, total;
 };
@@ -945,7 +1032,6 @@ int num_sms() {
   return n > 0 ? n : 148;
 }
 
-constexpr int kStatsCtasPerSm = 4;  // 3-stage 16 KB rings: 4 CTAs fit an SM
 
 // Work decomposition for these sizes; a pure function of the sizes and the SM
 // count, so repeated calls reduce in the same order (bit-reproducible).
@@ -972,10 +1058,15 @@ bool make_plan(int B, int K, int V, specdec_dtype dtype, int sms, Plan &pl) {
   // partial slots per row: the most CTAs whose tile ranges meet one row
   const long long minr = pl.tiles / pl.G1;  // shortest range
   pl.slots = (int)((tpr - 1 + minr - 1) / minr + 1);
-  const long long nr2 = (nvec_max + NT * 2 - 1) / (NT * 2);
-  pl.UR = ((long long)B * nr2 >= 2LL * sms) ? 2 : 1;
-  const long long nr = (nvec_max + (long long)NT * pl.UR - 1) / ((long long)NT * pl.UR);
+  // k_finish chunks: 32 lanes x kFinishUW vectors of the drawn row pair
+  const long long nr = (nvec_max + 32LL * kFinishUW - 1) / (32LL * kFinishUW);
   pl.nsr = (int)(nr > 0 ? nr : 1);
+  // chunks per CTA of k_finish: as many CTAs per sequence as keep the whole
+  // grid inside one wave (each CTA repeats the small acceptance step)
+  long long ncb = (long long)kFinishCtasPerSm * sms / (B > 0 ? B : 1);
+  if (ncb < 1) ncb = 1;
+  if (ncb > pl.nsr) ncb = pl.nsr;
+  pl.cpb = (int)((pl.nsr + ncb - 1) / ncb);
   if ((long long)B * pl.nsr > INT_MAX) return false;
   if ((long long)B * (K + 1) * (long long)V > (1LL << 56)) return false;
   size_t off = 0;
@@ -1082,10 +1173,10 @@ specdec_status launch_all(const void *tg, const void *dr, const int32_t *tok, co
   if (e != cudaSuccess) return SPECDEC_ECUDA;
   {
     LaunchTimer lt(KID_FINISH, st);
-    const unsigned g2 = (unsigned)((long long)B * pl.nsr);
-    auto kern = pl.UR == 2 ? k_finish<T, 2> : k_finish<T, 1>;
+    const unsigned g2 = (unsigned)((long long)B * ((pl.nsr + pl.cpb - 1) / pl.cpb));
+    auto kern = k_finish<T, kFinishUW>;
     e = launch_pdl(kern, g2, NT, st, t, d, tok, ua, ur, temp, K, (long long)V, pl.tpr, pl.tiles,
-                   pl.G1, pl.slots, pl.nsr,
+                   pl.G1, pl.slots, pl.nsr, pl.cpb,
                    (const Partial *)part, rp, cnt, out_tokens, out_n,
                    dbg ? dbg->row_max : nullptr, dbg ? dbg->row_sum : nullptr,
                    dbg ? dbg->p_x : nullptr, dbg ? dbg->q_x : nullptr, dbg ? dbg->Z : nullptr);
