@@ -67,9 +67,9 @@ def measured_peaks():
 
 
 def stored_traffic():
-    """dram bytes per launch of k_verify from the committed ncu capture,
+    """dram bytes per launch of k_row_stats from the committed ncu capture,
     valid only while the kernel source is unchanged since the capture."""
-    p = os.path.join(ROOT, "profiles", "k_verify_traffic.json")
+    p = os.path.join(ROOT, "profiles", "k_row_stats_traffic.json")
     src = os.path.join(ROOT, "speculative_sampling_b200", "csrc", "specdec.cu")
     try:
         with open(p) as f:
@@ -370,10 +370,10 @@ def run_cuda(args):
         "gpu_launches": launches,
     }
     if kern:
-        st_ms, st_n = kern["k_verify"]
+        st_ms, st_n = kern["k_row_stats"]
         avg = st_ms / max(st_n, 1)
         ach = floor / (avg * 1e-3) / 1e9
-        line["roofline"] = {"bound": "hbm", "kernel": "k_verify", "achieved": ach,
+        line["roofline"] = {"bound": "hbm", "kernel": "k_row_stats", "achieved": ach,
                             "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                             "frac": ach / peak, "traffic": stored_traffic(),
                             "algorithmic_bytes_per_launch": floor,

@@ -128,18 +128,10 @@ specdec_status specdec_verify_f32(const void *target_logits, const void *draft_l
  * (0 for invalid sizes). */
 size_t specdec_workspace_bytes(int B, int K, int V, specdec_dtype dtype);
 
-/* Prepare a caller-owned workspace for specdec_verify_ex: zeroes the counter
- * region at its start (asynchronously on `stream`).  Call it once after
- * allocating the workspace, and again whenever a different workspace_bytes is
- * to be passed with it.  Every completed call leaves the counter region zeroed,
- * so nothing has to be done between calls. */
-specdec_status specdec_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
-
 /* specdec_verify with a caller-owned workspace (device memory of at least
- * specdec_workspace_bytes bytes, 256-byte aligned, prepared once with
- * specdec_workspace_init and passed with the same workspace_bytes every time)
- * and optional diagnostics (dbg may be NULL).  Allocates nothing.  Calls that
- * share a workspace must not overlap on the device. */
+ * specdec_workspace_bytes bytes, 256-byte aligned; its contents need no
+ * initialisation) and optional diagnostics (dbg may be NULL).  Allocates
+ * nothing.  Calls that share a workspace must not overlap on the device. */
 specdec_status specdec_verify_ex(const void *target_logits, const void *draft_logits,
                                  const int32_t *draft_tokens, const float *u_accept,
                                  const float *u_resample, const float *temperature, int B,

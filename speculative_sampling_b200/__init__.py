@@ -29,7 +29,6 @@ _SIGS = {
     "specdec_verify_bf16": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P]),
     "specdec_verify_f32": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P]),
     "specdec_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
-    "specdec_workspace_init": (_I, [_P, ctypes.c_size_t, _P]),
     "specdec_verify_ex": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, ctypes.c_size_t, _P,
                                _P, _P, _P]),
     "specdec_verify_host": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P]),
@@ -106,10 +105,6 @@ def specdec_verify_f32(target, draft, tokens, u_accept, u_resample, temperature,
 
 def specdec_workspace_bytes(B, K, V, dtype) -> int:
     return lib().specdec_workspace_bytes(B, K, V, dtype)
-
-
-def specdec_workspace_init(workspace, workspace_bytes, stream) -> int:
-    return lib().specdec_workspace_init(workspace, workspace_bytes, stream)
 
 
 def specdec_verify_ex(target, draft, tokens, u_accept, u_resample, temperature, B, K, V, dtype,
@@ -194,10 +189,9 @@ def verify(target, draft, tokens, u_accept, u_resample, temperature, out_tokens=
     int32, u_accept [B,K] / u_resample [B] / temperature [B] float32.  Returns
     (out_tokens [B,K+1] int32, out_num_accepted [B] int32), written
     asynchronously on ``stream`` (default: torch's current stream).  With
-    ``workspace`` (a uint8 CUDA tensor of at least specdec_workspace_bytes
-    bytes, prepared once with workspace_init) or ``debug`` (dict of
-    preallocated tensors named as specdec_debug's fields) the call goes through
-    specdec_verify_ex."""
+    ``workspace`` (a uint8 CUDA tensor of specdec_workspace_bytes bytes) or
+    ``debug`` (dict of preallocated tensors named as specdec_debug's fields)
+    the call goes through specdec_verify_ex."""
     import torch
     B, K1, V = target.shape
     K = K1 - 1
@@ -225,7 +219,7 @@ def verify(target, draft, tokens, u_accept, u_resample, temperature, out_tokens=
         return out_tokens, out_num_accepted
     need = specdec_workspace_bytes(B, K, V, dt)
     if workspace is None:
-        workspace = torch.zeros((need,), dtype=torch.uint8, device=target.device)
+        workspace = torch.empty((need,), dtype=torch.uint8, device=target.device)
     dbg = None
     if debug is not None:
         d = _Debug()
@@ -237,16 +231,6 @@ def verify(target, draft, tokens, u_accept, u_resample, temperature, out_tokens=
                            out_tokens.data_ptr(), out_num_accepted.data_ptr(), stream)
     _chk(st, "specdec_verify_ex")
     return out_tokens, out_num_accepted
-
-
-def workspace_init(workspace, stream=None) -> None:
-    """Prepare a uint8 CUDA tensor for use as ``verify(..., workspace=...)``
-    (zeroes its counter region; needed once, not between calls)."""
-    import torch
-    if stream is None:
-        stream = torch.cuda.current_stream(workspace.device).cuda_stream
-    _chk(specdec_workspace_init(workspace.data_ptr(), workspace.numel(), stream),
-         "specdec_workspace_init")
 
 
 def verify_host(target, draft, tokens, u_accept, u_resample, temperature, out_tokens,

@@ -4,38 +4,23 @@
 // alpha(x) = min(1, p_target(x)/p_draft(x)), stop at the first rejection, draw
 // from max(0, p - q)/Z or from the bonus row; speculative decoding blog
 // "Speculative Decoding ... Llama 70B x2.4", section "The mathematical definition
-// from Leviathan et al.").  This file is the B200 implementation: one
-// persistent kernel, k_verify, runs the whole step.
+// from Leviathan et al.").  This file is the B200 implementation:
 //
-//   Work units, claimed one at a time from a global counter in a fixed order:
-//     statistics units  a few consecutive 16 KB tiles of one logit row; each
-//                       consumer warp leaves the (max, sum of 2^((z-max)c)) of
-//                       its share of the unit (split-V online softmax);
-//     residual units    one chunk of the drawn row pair of a sequence (target /
-//                       draft row n, or the target's bonus row K); each warp
-//                       leaves the sum of r(v) = St * max(0, p - q) over its
-//                       contiguous segment of the chunk.
-//   The residual units of sequence b follow the statistics units of sequence
-//   b + D, with the lag D sized so that b is normally decided (and its rows
-//   still in L2) by the time they are claimed.
-//   Tasks, run by the CTA that retires the last unit of a kind of a sequence
-//   (per-sequence arrival counters):
-//     ACCEPT  combine the row partials of the 2K+1 rows in fp64, gather
-//             p_i(x_i) and q_i(x_i), test u*q < p on K lanes, first rejection
-//             with __ballot_sync/__ffs, write the accepted prefix, publish the
-//             drawn row pair (a release flag the residual units wait on);
-//     DRAW    fp64 exclusive prefix over the segment sums, the segment holding
-//             u*Z, a block-wide rescan of that one segment, the drawn token.
-//
-// Inside a CTA: one producer thread streams the tiles of its units with
-// cp.async.bulk (the TMA bulk-copy engine; CTA-local copies, no multicast) into
-// an NSTAGE-deep shared-memory ring and schedules everything else (claims,
-// unit retirement, tasks) through the same ring; CW consumer warps fold tiles
-// in registers and run units and tasks in ring order.  Every wait (ring
-// barriers, the wait for a sequence to be decided, barriers among the consumer
-// warps) is bounded in wall-clock time: a wait that runs out sets
-// SPECDEC_ERR_TIMEOUT and the kernel winds down.  The grid is launched
-// cooperatively, so every CTA that another one may wait for is resident.
+//   k_row_stats  one pass over every logit row (B*(2K+1) rows of V): split-V
+//                online softmax statistics (row max m, sum of 2^((z-m)*c)) with
+//                16-byte non-temporal-in-L1 vector loads, a per-thread running
+//                max, warp-shuffle and shared-memory combines.  It streams the
+//                whole input once and is the HBM-bound kernel of the step.
+//   k_accept     one warp per sequence: combines the V-split partials of each of
+//                the 2K+1 rows in fp64, gathers p_i(x_i), q_i(x_i), tests
+//                u*q < p on K lanes and finds the first rejection with
+//                __ballot_sync/__ffs; writes the accepted prefix.
+//   k_resample   streams only the selected row pair (target/draft row n, or the
+//                target's bonus row K), forms r(v) = max(0, p - q) on the fly,
+//                reduces it per V-chunk; the last CTA of each sequence (atomic
+//                ticket, no waiting) takes the fp64 exclusive prefix over
+//                chunks, finds the chunk holding u*Z and rescans that one chunk
+//                with a block-wide fp64 scan to emit the drawn token.
 //
 // Arithmetic: logits are widened exactly to fp32.  Exponentials are
 // 2^((z - m) * c) with c = log2(e)/T carried as an fp32 pair (hi + lo, with
@@ -64,22 +49,22 @@
 
 namespace {
 
+constexpr int NT = 256;               // threads per CTA of the streaming kernels
+constexpr int NWARP = NT / 32;
 constexpr double kLog2e = 1.4426950408889634073599246810019;  // log2(e)
 constexpr unsigned FULL = 0xffffffffu;
 
 // ---------------------------------------------------------------------------
 // workspace records
 // ---------------------------------------------------------------------------
-struct __align__(16) Partial {  // one warp's share of a statistics unit
-  double s;                     // sum of 2^((z - m) c)
-  float m;                      // max
+struct __align__(16) Partial {  // one (row, V-split): max and sum of 2^((z-m)c)
+  double s;
+  float m;
   uint32_t pad;
 };
-struct __align__(16) SeqInfo {  // written by a sequence's ACCEPT task
-  double St, Sd;                // row sums (at the row max) of the drawn pair
-  float Mt, Md;                 // row maxima of the drawn pair
-  int n;                        // accepted length; -1 for an invalid sequence
-  int pad;
+struct __align__(16) ResPartial {  // one (sequence, V-chunk) of the drawn row(s)
+  double R;                        // sum of St * max(0, p - q)  (or of 2^((z-m)c), bonus)
+  double pad;
 };
 
 __device__ unsigned int g_error_flags;  // per device; read/cleared by the host
@@ -173,23 +158,36 @@ __device__ __forceinline__ float warp_max_nan(float v) {
   return v;
 }
 
+// ---------------------------------------------------------------------------
+// kernel 1: softmax statistics of every row
+// ---------------------------------------------------------------------------
+// The B*(2K+1) rows are cut into units: a unit is UT consecutive tiles of one
+// row; a tile is CW*32*U 16-byte vectors (16 KB for U = 4).  CTA g of a grid
+// of G handles units g, g+G, g+2G, ... so the grid sweeps the logits front to
+// back, sequence after sequence.
+//
+// Warp specialisation: one producer warp streams tiles with cp.async.bulk
+// (the TMA bulk-copy engine; plain CTA-local copies, no multicast) into an
+// NSTAGE-deep ring in shared memory, tracked by "full" / "empty" mbarriers;
+// CW consumer warps take a tile out of the ring (one 16-byte shared load per
+// vector), release the slot, and fold it into a per-thread (max, sum) in
+// registers.  A unit's setup (row pointer, alignment, log2(e)/T) and its
+// CTA combine are paid once per unit.  Per element the consumers spend one
+// exact bf16->fp32 unpack, one FMNMX for the tile max, three packed fp32x2
+// operations at half an issue slot each, one MUFU ex2 and half a packed add.
+// Every wait is bounded: a wait that runs out sets SPECDEC_ERR_TIMEOUT in the
+// device error word and the kernel winds down (the producer first waits, again
+// bounded, for the copies it has in flight).
 
-// ---------------------------------------------------------------------------
-// kernel geometry and synchronisation primitives
-// ---------------------------------------------------------------------------
 constexpr int CW = 8;               // consumer warps
 constexpr int NTC = CW * 32;        // consumer threads
 constexpr int NTS = NTC + 32;       // + one producer warp
 constexpr int NSTAGE = 3;           // depth of the shared-memory ring
-constexpr int NDONE = 8;            // units in flight per CTA (unit-done barriers)
-constexpr int NTASKQ = NDONE + 1;   // queued tasks per CTA
-constexpr int kCtasPerSm = 4;       // resident CTAs per SM the kernel is built for
-constexpr int UR = 4;               // vectors per lane and row in a residual segment
-constexpr int SV = 32 * UR;         // vectors per residual segment (one warp)
-constexpr int RV = CW * SV;         // vectors per residual unit and row
-constexpr int RMAX = 65;            // rows per sequence at K = 32
 constexpr unsigned long long kWaitNs = 2000000000ull;  // a wait gives up after 2 s
 constexpr unsigned kSuspendNs = 20000;  // longest sleep of one try_wait round
+constexpr int kStatsCtasPerSm = 4;  // resident CTAs per SM the sweep is sized for
+constexpr int kFinishUW = 4;        // vectors per lane in a k_finish chunk
+constexpr int kFinishCtasPerSm = 4; // k_finish grids fit one wave of this many CTAs per SM
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -219,17 +217,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, unsigned parity) {
       : "memory");
   return ok != 0;
 }
-// non-blocking test of the phase of the given parity
-__device__ __forceinline__ bool mbar_test(uint64_t *bar, unsigned parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
 __device__ __forceinline__ unsigned long long global_ns() {
   unsigned long long t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -255,24 +242,6 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, unsigned b
       ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
-// GPU-scope flag and counter operations between CTAs
-__device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
-  unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release(unsigned *p, unsigned v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ unsigned atom_add_acq_rel(unsigned *p, unsigned v) {
-  unsigned old;
-  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;"
-               : "=r"(old)
-               : "l"(p), "r"(v)
-               : "memory");
-  return old;
-}
-
 // pairs (x0, x1) of the 8 (bf16) or 4 (fp32) values of a 16-byte vector
 template <typename T>
 struct Pairs;
@@ -381,142 +350,264 @@ __device__ __forceinline__ void elem_fold(float x, RunStat &q, Scale c, float th
   q.acc.x += ex2(scaled(x + q.nr, c));
 }
 
-// ---------------------------------------------------------------------------
-// k_verify: the whole verify step in one persistent kernel
-// ---------------------------------------------------------------------------
-enum : int { E_STATS = 0, E_RES = 1, E_ACCEPT = 2, E_DRAW = 3, E_STOP = 4 };
-enum : int { F_FIRST = 1, F_LAST = 2, F_HEAD = 4, F_TAIL = 8 };
-
-// One ring entry, written by the producer before it arrives on the entry's
-// "full" barrier (which orders these stores before the consumers' reads).
-struct __align__(16) Entry {
-  int kind, b, j, flags;     // j: row of the sequence (statistics) or chunk (residual)
-  int nv, done, n, pad;      // nv: vectors in the tile; done: unit-done barrier; n: accepted length
-  long long unit, pad2;      // statistics unit: its partials are part[unit * CW + warp]
-  float chi, clo, thr, Mt;   // log2(e)/T of the sequence; residual: target row max
-  float Md, lhi, llo, pad3;  // residual: draft row max, St/Sd = lhi + llo
-};
-
-struct Params {
-  const void *target, *draft;
-  const int32_t *tokens;
-  const float *u_accept, *u_resample, *temperature;
-  int B, K;
+struct StatsGeom {
+  int K;
   long long V;
-  int tpr, tps, spr, nru, lag;  // tiles per row, tiles per unit, units per row, residual units
-  unsigned n_units;             // per sequence, lag in sequences; all units of the call
-  Partial *part;                // [B, 2K+1, spr, CW]
-  double *rpart;                // [B, nru, CW]   residual sums per segment
-  SeqInfo *seq;                 // [B]
-  unsigned *ctr;                // counters, see counter_words
-  int32_t *out_tokens, *out_n;
-  float *dbg_row_max;
-  double *dbg_row_sum, *dbg_px, *dbg_qx, *dbg_Z;
+  int tpr;          // tiles per row
+  long long tiles;  // rows * tpr
+  int slots;        // CTA slots per row (>= CTAs that can share one row)
 };
 
-// The counters are 32-bit words, all zero when a call starts and left zero
-// when it ends (the last CTA to exit clears them): [0] the unit claim counter,
-// [1] the CTA exit ticket, then per sequence b: [4+3b] statistics units
-// retired, [5+3b] residual units retired, [6+3b] the "decided" flag.
-constexpr int kCtrHead = 4;
-__host__ __device__ __forceinline__ long long counter_words(long long B) {
-  return kCtrHead + 3 * B;
+// CTA g of G owns tiles [g*T/G, (g+1)*T/G); the owner of tile t is then
+// floor(((t+1)*G - 1) / T).  Both the statistics kernel and the combine in
+// k_finish use these to name a row's partials: CTA slot = owner - first owner,
+// and each of the CW consumer warps of a CTA writes its own partial.
+__host__ __device__ __forceinline__ long long tile_begin(long long g, long long G, long long T) {
+  return g * T / G;
+}
+__host__ __device__ __forceinline__ long long tile_owner(long long t, long long G, long long T) {
+  return ((t + 1) * G - 1) / T;
 }
 
-// The work list: S statistics units per sequence (2K+1 rows x spr units),
-// NR residual units per sequence; the residual units of sequence b come right
-// after the statistics units of sequence b + D (or at the end of the list).
-struct UnitRef {
-  int kind;
-  long long b, k;  // sequence; statistics unit within it, or residual chunk
-};
-__host__ __device__ __forceinline__ UnitRef decode_unit(long long u, long long B, long long S,
-                                                      long long NR, long long D) {
-  UnitRef r;
-  const long long E1 = D * S, E2 = E1 + (B - D) * (S + NR);
-  if (u < E1) {
-    r.kind = E_STATS;
-    r.b = u / S;
-    r.k = u - r.b * S;
-  } else if (u < E2) {
-    const long long m = (u - E1) / (S + NR), k = (u - E1) - m * (S + NR);
-    if (k < S) {
-      r.kind = E_STATS;
-      r.b = D + m;
-      r.k = k;
-    } else {
-      r.kind = E_RES;
-      r.b = m;
-      r.k = k - S;
+// The current row of a CTA's tile walk.  Rows are numbered b*(2K+1) + j with
+// j = 0..K the target rows and j = K+1..2K the draft rows of sequence b; the
+// cursor steps row by row without divisions.
+template <typename T>
+struct RowCursor {
+  const T *p;
+  const uint4 *pv;
+  long long row, b, nvec;
+  int j, ti, head;
+  __device__ __forceinline__ void point(const T *target, const T *draft, const StatsGeom &g) {
+    constexpr int VEC = Dt<T>::VEC;
+    p = (j <= g.K) ? target + (b * (g.K + 1) + j) * g.V
+                   : draft + (b * g.K + (j - g.K - 1)) * g.V;
+    head = row_head(p, g.V);
+    nvec = (g.V - head) / VEC;
+    pv = reinterpret_cast<const uint4 *>(p + head);
+  }
+  __device__ __forceinline__ void start(const T *target, const T *draft, const StatsGeom &g,
+                                        long long t) {
+    const int R = 2 * g.K + 1;
+    row = t / g.tpr;
+    ti = (int)(t - row * g.tpr);
+    b = row / R;
+    j = (int)(row - b * R);
+    point(target, draft, g);
+  }
+  __device__ __forceinline__ void next_row(const T *target, const T *draft, const StatsGeom &g) {
+    ++row;
+    ti = 0;
+    if (++j == 2 * g.K + 1) {
+      j = 0;
+      ++b;
     }
-  } else {
-    const long long v = u - E2, m = v / NR;
-    r.kind = E_RES;
-    r.b = B - D + m;
-    r.k = v - m * NR;
+    point(target, draft, g);
   }
-  return r;
-}
-
-struct Smem {
-  uint64_t full[NSTAGE], empty[NSTAGE], done[NDONE], cbar;
-  Entry ent[NSTAGE];
-  float sM[RMAX];
-  double sS[RMAX];
-  double scan[CW];
-  double s_base;
-  int abort, last_cta;
-  int s_seg, s_y, s_lastpos;
 };
 
-// Barrier of the CW consumer warps on an mbarrier, bounded like every other
-// wait; false when it ran out or the CTA is winding down (the caller stops).
-__device__ __forceinline__ bool csync(Smem &sm, unsigned &cph) {
-  if (*(volatile int *)&sm.abort) return false;
-  __syncwarp();
-  if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.cbar);
-  const bool ok = __all_sync(FULL, mbar_wait(&sm.cbar, cph));
-  cph ^= 1u;
-  if (!ok && (threadIdx.x & 31) == 0) atomicExch(&sm.abort, 1);
-  return ok;
+template <typename T, int U>
+__global__ void __launch_bounds__(NTS, kStatsCtasPerSm) k_row_stats(const T *__restrict__ target,
+                                                   const T *__restrict__ draft,
+                                                   const float *__restrict__ temperature,
+                                                   StatsGeom g, Partial *__restrict__ part,
+                                                   unsigned *__restrict__ tickets, int B) {
+  constexpr int VEC = Dt<T>::VEC;
+  constexpr long long TV = (long long)NTC * U;  // vectors per tile
+  constexpr unsigned TILE_BYTES = (unsigned)TV * 16u;
+  extern __shared__ __align__(128) unsigned char ring[];  // NSTAGE * TILE_BYTES
+  __shared__ __align__(8) uint64_t full[NSTAGE], empty[NSTAGE];
+  __shared__ int s_abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long G = gridDim.x;
+  const long long t0 = tile_begin(blockIdx.x, G, g.tiles);
+  const long long t1 = tile_begin(blockIdx.x + 1, G, g.tiles);
+
+  // the arrival tickets of k_finish (which runs after this kernel) start at 0
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < B; i += blockDim.x) tickets[i] = 0u;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NSTAGE; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], CW);
+    }
+    s_abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (t0 >= t1) return;
+
+  // The CTA's tiles [t0, t1) are walked as row segments: the tiles of one row
+  // that fall in the range.  Inside a segment the full tiles come first (no
+  // per-element predicates), then at most one partial tile.
+  const long long row_first = t0 / g.tpr, row_last = (t1 - 1) / g.tpr;
+
+  if (warp == CW) {  // ---------------- producer warp ----------------
+    if (lane != 0) return;
+    unsigned it = 0, ph = 0;  // copies issued; phase parity of the current ring pass
+    int st = 0;               // ring slot of the next copy
+    RowCursor<T> rc;
+    rc.start(target, draft, g, t0);
+    for (long long row = row_first; row <= row_last; ++row) {
+      if (row != row_first) rc.next_row(target, draft, g);
+      const int tb = (row == row_first) ? (int)(t0 - row * g.tpr) : 0;
+      const int te = (row == row_last) ? (int)(t1 - row * g.tpr) : g.tpr;
+      for (int ti = tb; ti < te; ++ti) {
+        const long long v0 = (long long)ti * TV;
+        const long long v1 = (v0 + TV < rc.nvec) ? v0 + TV : rc.nvec;
+        if (v0 >= v1) break;  // the rest of the row is its scalar tail
+        if (*(volatile int *)&s_abort || !mbar_wait(&empty[st], ph ^ 1u)) {
+          atomicExch(&s_abort, 1);
+          goto drain;
+        }
+        const unsigned bytes = (unsigned)(v1 - v0) * 16u;
+        mbar_arrive_tx(&full[st], bytes);
+        bulk_load(ring + (size_t)st * TILE_BYTES, rc.pv + v0, bytes, &full[st]);
+        ++it;
+        if (++st == NSTAGE) {
+          st = 0;
+          ph ^= 1u;
+        }
+      }
+    }
+  drain:
+    // The CTA must not retire with copies in flight: wait (bounded) until the
+    // last copy issued into each slot has landed.
+    for (unsigned k = 0; k < NSTAGE && k < it; ++k) {
+      const unsigned j = it - 1 - k;
+      mbar_wait(&full[j % NSTAGE], (j / NSTAGE) & 1u);
+    }
+    return;
+  }
+
+  // ---------------- consumer warps ----------------
+  // No CTA-wide barrier inside the walk: each warp folds its share of every
+  // tile and, at the end of a row segment, reduces its lanes and writes its own
+  // partial.  After an abort the waits and the arithmetic are skipped (every
+  // warp still walks the same tiles).
+  unsigned ph = 0;  // phase parity of the current ring pass
+  int st = 0;       // ring slot of the next tile
+  RowCursor<T> rc;
+  rc.start(target, draft, g, t0);
+  Scale c = make_scale(kLog2e / (double)__ldg(temperature + rc.b));
+  float thr = 64.0f / c.hi;
+  // temperature of the sequence after this one, fetched a row ahead
+  float T_next = (rc.b + 1 < B) ? __ldg(temperature + rc.b + 1) : 1.0f;
+  for (long long row = row_first; row <= row_last; ++row) {
+    if (row != row_first) {
+      const bool new_seq = (rc.j == 2 * g.K);
+      rc.next_row(target, draft, g);
+      if (new_seq) {
+        c = make_scale(kLog2e / (double)T_next);
+        thr = 64.0f / c.hi;
+        T_next = (rc.b + 1 < B) ? __ldg(temperature + rc.b + 1) : 1.0f;
+      }
+    }
+    const int tb = (row == row_first) ? (int)(t0 - row * g.tpr) : 0;
+    const int te = (row == row_last) ? (int)(t1 - row * g.tpr) : g.tpr;
+    const long long full_tiles = rc.nvec / TV;  // tiles with all TV vectors
+    const int tf = (int)((long long)te < full_tiles ? te : full_tiles);
+    RunStat q;
+    runstat_init(q);
+    // full tiles
+    for (int ti = tb; ti < tf; ++ti) {
+      bool have = false;
+      if (!*(volatile int *)&s_abort) {
+        have = __all_sync(FULL, mbar_wait(&full[st], ph));
+        if (!have && lane == 0) atomicExch(&s_abort, 1);
+      }
+      const uint4 *tile = reinterpret_cast<const uint4 *>(ring + (size_t)st * TILE_BYTES);
+      if (++st == NSTAGE) {
+        st = 0;
+        ph ^= 1u;
+      }
+      if (!have) continue;
+      uint4 v[U];
+#pragma unroll
+      for (int k = 0; k < U; ++k) v[k] = tile[k * NTC + threadIdx.x];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st == 0 ? NSTAGE - 1 : st - 1]);
+#pragma unroll
+      for (int k = 0; k < U; ++k) vec_fold<T>(v[k], q, c, thr);
+    }
+    // at most one partial tile (the row's last vectors)
+    const int tpb = tb > tf ? tb : tf;
+    if (tpb < te && (long long)tpb * TV < rc.nvec) {
+      const long long nv = rc.nvec - (long long)tpb * TV;
+      bool have = false;
+      if (!*(volatile int *)&s_abort) {
+        have = __all_sync(FULL, mbar_wait(&full[st], ph));
+        if (!have && lane == 0) atomicExch(&s_abort, 1);
+      }
+      const uint4 *tile = reinterpret_cast<const uint4 *>(ring + (size_t)st * TILE_BYTES);
+      const int cur = st;
+      if (++st == NSTAGE) {
+        st = 0;
+        ph ^= 1u;
+      }
+      if (have) {
+        uint4 v[U];
+#pragma unroll
+        for (int k = 0; k < U; ++k) {
+          const int vi = k * NTC + threadIdx.x;
+          v[k] = (vi < nv) ? tile[vi] : Dt<T>::neg_inf();
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[cur]);
+#pragma unroll
+        for (int k = 0; k < U; ++k) vec_fold<T>(v[k], q, c, thr);
+      }
+    }
+    // scalar head / tail of the row when this CTA holds its first / last tile
+    if (tb == 0 && (int)threadIdx.x < rc.head)
+      elem_fold(Dt<T>::load(rc.p + threadIdx.x), q, c, thr);
+    if (te == g.tpr) {
+      const long long tt = rc.head + rc.nvec * VEC + threadIdx.x;
+      if (tt < g.V) elem_fold(Dt<T>::load(rc.p + tt), q, c, thr);
+    }
+    // this warp's partial: lanes combined in fp64 with shuffles
+    const float m = q.mt;
+    const float sl = runstat_sum_at_max(q, c);
+    const float mw = warp_max_nan(m);
+    double sw = (m == -INFINITY) ? 0.0 : (double)sl * (double)ex2(scaled(m - mw, c));
+    sw = warp_sum(sw);
+    if (lane == 0) {
+      const long long slot = (long long)blockIdx.x - tile_owner(row * g.tpr, G, g.tiles);
+      Partial out;
+      out.s = sw;
+      out.m = mw;
+      out.pad = 0;
+      part[(row * g.slots + slot) * CW + warp] = out;
+    }
+  }
 }
 
-// Exclusive prefix sum of one double per consumer thread, in thread order
-// (fixed association); `total` receives the sum over all of them.
-__device__ __forceinline__ bool cta_excl_scan(double v, double &excl, double &total, Smem &sm,
-                                              unsigned &cph) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  double incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const double y = __shfl_up_sync(FULL, incl, o);
-    if (lane >= o) incl += y;
-  }
-  double ex = __shfl_up_sync(FULL, incl, 1);
-  if (lane == 0) ex = 0.0;
-  if (!csync(sm, cph)) return false;  // earlier readers of sm.scan are done
-  if (lane == 31) sm.scan[warp] = incl;
-  if (!csync(sm, cph)) return false;
-  double base = 0.0, tot = 0.0;
-#pragma unroll
-  for (int w = 0; w < CW; ++w) {
-    if (w < warp) base += sm.scan[w];
-    tot += sm.scan[w];
-  }
-  excl = base + ex;
-  total = tot;
-  return true;
-}
+// ---------------------------------------------------------------------------
+// kernel 2: accept test + residual / bonus draw ("finish")
+// ---------------------------------------------------------------------------
+// Grid: B sequences x nsr V-chunks.  Every CTA of sequence b first repeats the
+// (small) acceptance step for b: it combines the V-split partials of the 2K+1
+// rows in fp64, gathers p_i(x_i) and q_i(x_i) (fp64 exp2 of exact logits),
+// tests u*q < p on K lanes and finds the first rejection n with __ballot_sync /
+// __ffs.  Chunk 0 writes the accepted prefix.  Then each CTA streams its chunk
+// of the drawn row pair (target/draft row n, or the target's row K for the
+// bonus), forming r(v) = St * max(0, p - q) = max(0, e_t - (St/Sd) e_d) on the
+// fly (or e_t for the bonus), and adds it up in fp64.  The last CTA of the
+// sequence to finish (atomic arrival ticket; nothing waits) draws: block scan
+// of the chunk sums in fp64, the chunk holding u*Z, then a block scan over
+// that chunk with the weights kept in registers, first crossing wins.  When
+// the residual mass is below 2^-64 the fp32 weights have run out of range and
+// the draw is redone in fp64 over the whole row pair.
 
-// The drawn row pair of a sequence: r = St * max(0, p - q) = max(0, e_t -
-// (St/Sd) e_d) with e = 2^((z - m)c), or e_t for the bonus row.  The same
-// inlined arithmetic serves the segment sums and the rescan, so both see
-// bit-identical per-element weights.
 struct DrawRow {
   float Mt, Md, lhi, llo;
   Scale c;
   bool bonus;
 };
+
+// r = St * max(0, p - q) = max(0, e_t - (St/Sd) e_d) with e = 2^((z - m)c)
+// (or e_t for the bonus row).  The same inlined arithmetic serves the chunk
+// sums and the rescan, so both see bit-identical per-element weights.
 __device__ __forceinline__ float res_weight(float zt, float zd, const DrawRow &d) {
   const float et = ex2(scaled(zt - d.Mt, d.c));
   if (d.bonus) return et;
@@ -526,16 +617,29 @@ __device__ __forceinline__ float res_weight(float zt, float zd, const DrawRow &d
   return t2 > 0.0f ? t2 : 0.0f;
 }
 
-// Element range [lo, hi) of residual segment s (of NS) of a row whose first
-// 16-byte boundary is `head` elements in and which holds nvec whole vectors:
-// segment s takes vectors [s*SV, (s+1)*SV); segment 0 also the head, the last
-// segment also the scalar tail.
-template <int VEC>
-__device__ __forceinline__ void segment_range(int s, int NS, int head, long long nvec, long long V,
-                                              long long &lo, long long &hi) {
-  const long long a = (long long)s * SV, e = (long long)(s + 1) * SV;
-  lo = (s == 0) ? 0 : head + (a < nvec ? a : nvec) * VEC;
-  hi = (s == NS - 1) ? V : head + (e < nvec ? e : nvec) * VEC;
+// Block-wide exclusive prefix sum of one double per thread, in thread order
+// (fixed association); `total` receives the block sum.  All threads call it.
+__device__ __forceinline__ double block_excl_scan(double v, double &total) {
+  __shared__ double sm[NWARP];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  double incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double y = __shfl_up_sync(FULL, incl, o);
+    if (lane >= o) incl += y;
+  }
+  double excl = __shfl_up_sync(FULL, incl, 1);
+  if (lane == 0) excl = 0.0;
+  __syncthreads();  // a previous call may still be reading sm
+  if (lane == 31) sm[warp] = incl;
+  __syncthreads();
+  double base = 0.0, tot = 0.0;
+  for (int w = 0; w < NWARP; ++w) {
+    if (w < warp) base += sm[w];
+    tot += sm[w];
+  }
+  total = tot;
+  return base + excl;
 }
 
 // fp64 probability of one logit: 2^((z - M) c) / S
@@ -544,16 +648,15 @@ __device__ __forceinline__ double prob64(const T *row, long long v, float M, dou
   return exp2(((double)Dt<T>::load(row + v) - (double)M) * c64) / S;
 }
 
-// Inverse-CDF draw from max(0, p - q) entirely in fp64 by the consumer warps
-// (contiguous ranges per thread, block scan, first crossing).  If the fp64
+// Inverse-CDF draw from max(0, p - q) entirely in fp64 by the whole CTA
+// (contiguous segments per thread, block scan, first crossing).  If the fp64
 // residual is zero as well, draws from p (as the oracle does).  Used only when
-// the fp32 residual weights have run out of range.  sm.s_y / sm.s_lastpos
-// must hold INT_MAX / -1 on entry.
+// the fp32 residual weights have run out of range.
 template <typename T>
-__device__ __noinline__ bool draw_exact64(const T *pt, const T *pd, long long V, float Mt,
-                                          double St, float Md, double Sd, double c64, double u,
-                                          Smem &sm, unsigned &cph, int &y, double &Z) {
-  const long long E = (V + NTC - 1) / NTC;
+__device__ __noinline__ int draw_exact64(const T *pt, const T *pd, long long V, float Mt,
+                                         double St, float Md, double Sd, double c64, double u,
+                                         int *s_y, int *s_lastpos, double *dbg_Z) {
+  const long long E = (V + NT - 1) / NT;
   const long long e0 = (long long)threadIdx.x * E < V ? (long long)threadIdx.x * E : V;
   const long long e1 = (e0 + E < V) ? e0 + E : V;
   double sr = 0.0, sp = 0.0;
@@ -563,10 +666,11 @@ __device__ __noinline__ bool draw_exact64(const T *pt, const T *pd, long long V,
     sr += (p - q > 0.0) ? p - q : 0.0;
     sp += p;
   }
-  double xr, Zr, xp, Zp;
-  if (!cta_excl_scan(sr, xr, Zr, sm, cph) || !cta_excl_scan(sp, xp, Zp, sm, cph)) return false;
+  double Zr, Zp;
+  const double xr = block_excl_scan(sr, Zr);
+  const double xp = block_excl_scan(sp, Zp);
   const bool use_p = !(Zr > 0.0);
-  Z = use_p ? Zp : Zr;
+  const double Z = use_p ? Zp : Zr;
   const double t = u * Z;
   double C = use_p ? xp : xr;
   int last = -1;
@@ -578,95 +682,109 @@ __device__ __noinline__ bool draw_exact64(const T *pt, const T *pd, long long V,
     if (x > 0.0) last = (int)v;
     C += x;
     if (!found && C > t) {
-      atomicMin(&sm.s_y, (int)v);
+      atomicMin(s_y, (int)v);
       found = true;
     }
   }
-  if (last >= 0) atomicMax(&sm.s_lastpos, last);
-  if (!csync(sm, cph)) return false;
-  y = (sm.s_y != INT_MAX) ? sm.s_y : (sm.s_lastpos >= 0 ? sm.s_lastpos : 0);
-  return true;
+  if (last >= 0) atomicMax(s_lastpos, last);
+  __syncthreads();
+  const int y = (*s_y != INT_MAX) ? *s_y : (*s_lastpos >= 0 ? *s_lastpos : 0);
+  if (threadIdx.x == 0 && dbg_Z) *dbg_Z = Z;
+  return y;
 }
 
-// ---- ACCEPT: decide sequence b (all consumer warps) ----
-template <typename T>
-__device__ __noinline__ void accept_task(const Params &p, int b, Smem &sm, unsigned &cph) {
+template <typename T, int UW>
+__global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
+    const T *__restrict__ target, const T *__restrict__ draft,
+    const int32_t *__restrict__ tokens, const float *__restrict__ u_accept,
+    const float *__restrict__ u_resample, const float *__restrict__ temperature, int K,
+    long long V, int tpr, long long tiles, long long G1, int slots, int nsr, int cpb,
+    const Partial *__restrict__ part,
+    ResPartial *__restrict__ rpart, unsigned *__restrict__ counters,
+    int32_t *__restrict__ out_tokens, int32_t *__restrict__ out_n,
+    float *__restrict__ dbg_row_max, double *__restrict__ dbg_row_sum,
+    double *__restrict__ dbg_px, double *__restrict__ dbg_qx, double *__restrict__ dbg_Z) {
+  constexpr int VEC = Dt<T>::VEC;
+  constexpr long long CHV = 32LL * UW;                 // vectors per (warp-)chunk
+  constexpr long long CH = CHV * VEC;                  // elements per chunk
+  constexpr int EMAX = (int)((CH + 2 * VEC + NT - 1) / NT);  // rescan elements per thread
+  __shared__ float sM[65];
+  __shared__ double sS[65];
+  __shared__ int s_n, s_last, s_mode, s_chunk, s_y, s_lastpos;
+  __shared__ double s_base, s_t;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int K = p.K, R = 2 * K + 1;
-  const long long V = p.V;
-  const T *target = static_cast<const T *>(p.target);
-  const T *draft = static_cast<const T *>(p.draft);
-  const float Tf = __ldg(p.temperature + b);
+  const int ncb = (nsr + cpb - 1) / cpb;  // CTAs per sequence
+  const long long b = (long long)blockIdx.x / ncb;
+  const int cb = (int)((long long)blockIdx.x - b * ncb);  // this CTA: chunks cb*cpb ...
+  const int R = 2 * K + 1;
+
+  // ---- inputs of this call (independent of the statistics kernel) ----
+  const float Tf = __ldg(temperature + b);
   const bool t_ok = isfinite(Tf) && Tf > 0.0f;
   const double c64 = kLog2e / (double)Tf;
-  // the gathers first, so their latency overlaps the combine
   int x = 0;
   bool x_ok = true;
   float zt_x = 0.f, zd_x = 0.f, u = 0.f;
   if (warp == 0 && lane < K) {
-    x = __ldg(p.tokens + (long long)b * K + lane);
+    x = __ldg(tokens + b * K + lane);
     x_ok = (x >= 0) && ((long long)x < V);
-    u = __ldg(p.u_accept + (long long)b * K + lane);
+    u = __ldg(u_accept + b * K + lane);
     if (x_ok) {
-      zt_x = Dt<T>::load(target + ((long long)b * (K + 1) + lane) * V + x);
-      zd_x = Dt<T>::load(draft + ((long long)b * K + lane) * V + x);
+      zt_x = Dt<T>::load(target + (b * (K + 1) + lane) * V + x);
+      zd_x = Dt<T>::load(draft + (b * K + lane) * V + x);
     }
   }
-  // combine the partials of each row in fp64 (written by other CTAs in this
-  // call: read through L2)
-  const int np = p.spr * CW;
-  for (int r = warp; r < R; r += CW) {
-    const Partial *P = p.part + ((long long)b * R + r) * np;
-    constexpr int PL = 4;  // partials per lane kept in registers
-    double ps[PL];
-    float pm[PL];
-    float m = -INFINITY;
-#pragma unroll
-    for (int k = 0; k < PL; ++k) {
-      const int s = lane + 32 * k;
-      ps[k] = 0.0;
-      pm[k] = -INFINITY;
-      if (s < np) {
-        ps[k] = __ldcg(&P[s].s);
-        pm[k] = __ldcg(&P[s].m);
-      }
-      m = fmax_nan(m, pm[k]);
-    }
-    for (int s = lane + 32 * PL; s < np; s += 32) m = fmax_nan(m, __ldcg(&P[s].m));
+  const float ures = __ldg(u_resample + b);
+  cudaGridDependencySynchronize();  // the row statistics are complete from here on
+
+  // ---- combine the V-split partials of every row (fp64) ----
+  for (int r = warp; r < R; r += NWARP) {
+    const long long row = b * R + r;
+    const Partial *P = part + row * slots * CW;
+    // partials of the CTAs of the statistics sweep that hold tiles of this
+    // row, in order, CW consumer warps each
+    const int nslot = (int)(tile_owner(row * tpr + tpr - 1, G1, tiles) -
+                            tile_owner(row * tpr, G1, tiles) + 1) * CW;
+    // first 32 partials in registers (one load per lane), the rest streamed
+    Partial p0;
+    p0.m = -INFINITY;
+    p0.s = 0.0;
+    if (lane < nslot) p0 = P[lane];
+    float m = p0.m;
+    for (int s = lane + 32; s < nslot; s += 32) m = fmaxf(m, P[s].m);
     m = warp_max_nan(m);
-    double acc = 0.0;
-#pragma unroll
-    for (int k = 0; k < PL; ++k)
-      acc += (pm[k] == -INFINITY) ? ps[k] : ps[k] * exp2(((double)pm[k] - (double)m) * c64);
-    for (int s = lane + 32 * PL; s < np; s += 32) {
-      const float ms = __ldcg(&P[s].m);
-      const double ss = __ldcg(&P[s].s);
-      acc += (ms == -INFINITY) ? ss : ss * exp2(((double)ms - (double)m) * c64);
+    double acc = (lane < nslot)
+                     ? ((p0.m == -INFINITY) ? p0.s : p0.s * exp2(((double)p0.m - (double)m) * c64))
+                     : 0.0;
+    for (int s = lane + 32; s < nslot; s += 32) {
+      const Partial ps = P[s];
+      acc += (ps.m == -INFINITY) ? ps.s : ps.s * exp2(((double)ps.m - (double)m) * c64);
     }
     acc = warp_sum(acc);
     if (lane == 0) {
-      sm.sM[r] = m;
-      sm.sS[r] = acc;
-      if (p.dbg_row_max) p.dbg_row_max[(long long)b * R + r] = m;
-      if (p.dbg_row_sum) p.dbg_row_sum[(long long)b * R + r] = acc;
+      sM[r] = m;
+      sS[r] = acc;
+      if (cb == 0 && dbg_row_max) dbg_row_max[b * R + r] = m;
+      if (cb == 0 && dbg_row_sum) dbg_row_sum[b * R + r] = acc;
     }
   }
-  if (!csync(sm, cph)) return;
+  __syncthreads();
 
+  // ---- acceptance test and first rejection (warp 0) ----
   if (warp == 0) {
     // a timed-out wait in this call (or an earlier, unacknowledged one) makes
     // every sequence invalid rather than silently wrong
     const bool timed_out = (*(volatile unsigned *)&g_error_flags & SPECDEC_ERR_TIMEOUT) != 0;
     bool rows_ok = true;
     for (int r = lane; r < R; r += 32)
-      rows_ok = rows_ok && isfinite(sm.sM[r]) && isfinite(sm.sS[r]) && sm.sS[r] > 0.0;
+      rows_ok = rows_ok && isfinite(sM[r]) && isfinite(sS[r]) && sS[r] > 0.0;
     rows_ok = __all_sync(FULL, rows_ok) && !timed_out;
     bool acc_i = false;
-    double pp = 0.0, qq = 0.0;
+    double p = 0.0, q = 0.0;
     if (lane < K && x_ok && rows_ok && t_ok) {
-      pp = exp2(((double)zt_x - (double)sm.sM[lane]) * c64) / sm.sS[lane];
-      qq = exp2(((double)zd_x - (double)sm.sM[K + 1 + lane]) * c64) / sm.sS[K + 1 + lane];
-      acc_i = (double)u * qq < pp;
+      p = exp2(((double)zt_x - (double)sM[lane]) * c64) / sS[lane];
+      q = exp2(((double)zd_x - (double)sM[K + 1 + lane]) * c64) / sS[K + 1 + lane];
+      acc_i = (double)u * q < p;
     }
     const unsigned bad_x = __ballot_sync(FULL, lane < K && !x_ok);
     const unsigned accm = __ballot_sync(FULL, lane < K && acc_i);
@@ -674,200 +792,196 @@ __device__ __noinline__ void accept_task(const Params &p, int b, Smem &sm, unsig
     const unsigned kmask = (K >= 32) ? FULL : ((1u << K) - 1u);
     const unsigned rej = ~accm & kmask;
     const int n = seq_ok ? (rej ? __ffs(rej) - 1 : K) : -1;
-    int32_t *ot = p.out_tokens + (long long)b * (K + 1);
-    if (!seq_ok) {
-      for (int i = lane; i <= K; i += 32) ot[i] = -1;
-    } else {
-      if (lane < n) ot[lane] = x;
-      for (int i = n + 1 + lane; i <= K; i += 32) ot[i] = -1;
-      if (lane < K && lane <= n) {
-        if (p.dbg_px) p.dbg_px[(long long)b * K + lane] = pp;
-        if (p.dbg_qx) p.dbg_qx[(long long)b * K + lane] = qq;
-      }
-    }
-    if (lane == 0) {
-      p.out_n[b] = n;
+    if (lane == 0) s_n = n;
+    if (cb == 0) {
+      int32_t *ot = out_tokens + b * (K + 1);
       if (!seq_ok) {
-        unsigned f = 0;
-        if (!t_ok) f |= SPECDEC_ERR_TEMPERATURE;
-        if (bad_x) f |= SPECDEC_ERR_TOKEN;
-        if (!rows_ok && !timed_out) f |= SPECDEC_ERR_LOGITS;
-        if (f) atomicOr(&g_error_flags, f);
+        for (int i = lane; i <= K; i += 32) ot[i] = -1;
+      } else {
+        if (lane < n) ot[lane] = x;
+        for (int i = n + 1 + lane; i <= K; i += 32) ot[i] = -1;
+        if (lane < K && lane <= n) {
+          if (dbg_px) dbg_px[b * K + lane] = p;
+          if (dbg_qx) dbg_qx[b * K + lane] = q;
+        }
       }
-      SeqInfo si;
-      si.n = n;
-      si.pad = 0;
-      si.Mt = n >= 0 ? sm.sM[n] : 0.f;
-      si.St = n >= 0 ? sm.sS[n] : 1.0;
-      si.Md = (n >= 0 && n < K) ? sm.sM[K + 1 + n] : 0.f;
-      si.Sd = (n >= 0 && n < K) ? sm.sS[K + 1 + n] : 1.0;
-      p.seq[b] = si;
-      // publish: the residual units of b wait for this flag
-      st_release(p.ctr + kCtrHead + 3LL * b + 2, 1u);
-    }
-  }
-  csync(sm, cph);  // sM / sS are free again
-}
-
-// ---- residual unit: one warp's segment sum of the drawn row pair ----
-template <typename T>
-__device__ __forceinline__ double residual_sum(const Params &p, int b, int chunk, int n,
-                                               const DrawRow &d) {
-  constexpr int VEC = Dt<T>::VEC;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (n < 0) return 0.0;
-  const int K = p.K;
-  const long long V = p.V;
-  const T *pt = static_cast<const T *>(p.target) + ((long long)b * (K + 1) + n) * V;
-  const T *pd = d.bonus ? pt : static_cast<const T *>(p.draft) + ((long long)b * K + n) * V;
-  const int head = row_head(pt, V);
-  const long long nvec = (V - head) / VEC;
-  const int NS = p.nru * CW;
-  const int s = chunk * CW + warp;
-  float rs = 0.f;
-  if (d.bonus || row_head(pd, V) == head) {
-    const uint4 *vt = reinterpret_cast<const uint4 *>(pt + head);
-    const uint4 *vd = reinterpret_cast<const uint4 *>(pd + head);
-    const long long v0 = (long long)s * SV;
-    uint4 at[UR], ad[UR];
-#pragma unroll
-    for (int k = 0; k < UR; ++k) {
-      const long long vi = v0 + k * 32 + lane;
-      at[k] = vi < nvec ? __ldg(vt + vi) : make_uint4(0, 0, 0, 0);
-      ad[k] = (vi < nvec && !d.bonus) ? __ldg(vd + vi) : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int k = 0; k < UR; ++k) {
-      if (v0 + k * 32 + lane < nvec) {
-        float xt[VEC], xd[VEC];
-        Dt<T>::unpack(at[k], xt);
-        Dt<T>::unpack(ad[k], xd);
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) rs += res_weight(xt[e], xd[e], d);
+      if (lane == 0) {
+        out_n[b] = n;
+        if (!seq_ok) {
+          unsigned f = 0;
+          if (!t_ok) f |= SPECDEC_ERR_TEMPERATURE;
+          if (bad_x) f |= SPECDEC_ERR_TOKEN;
+          if (!rows_ok) f |= SPECDEC_ERR_LOGITS;
+          atomicOr(&g_error_flags, f);
+        }
       }
     }
-    if (s == 0 && lane < head)
-      rs += res_weight(Dt<T>::load(pt + lane), d.bonus ? 0.f : Dt<T>::load(pd + lane), d);
-    if (s == NS - 1) {
-      const long long tt = head + nvec * VEC + lane;
-      if (lane < VEC && tt < V)
-        rs += res_weight(Dt<T>::load(pt + tt), d.bonus ? 0.f : Dt<T>::load(pd + tt), d);
-    }
-  } else {  // rows of different alignment: scalar loads over the segment
-    long long lo, hi;
-    segment_range<VEC>(s, NS, head, nvec, V, lo, hi);
-    for (long long v = lo + lane; v < hi; v += 32)
-      rs += res_weight(Dt<T>::load(pt + v), Dt<T>::load(pd + v), d);
   }
-  return warp_sum((double)rs);
-}
+  __syncthreads();
+  const int n = s_n;
+  if (n < 0) return;  // invalid sequence (the same for every CTA of it)
 
-// ---- DRAW: the drawn token of sequence b (all consumer warps) ----
-template <typename T>
-__device__ __noinline__ void draw_task(const Params &p, int b, Smem &sm, unsigned &cph) {
-  constexpr int VEC = Dt<T>::VEC;
-  constexpr int EMAX = (SV * VEC + 2 * VEC + NTC - 1) / NTC;  // rescan elements per thread
-  const int tid = threadIdx.x;
-  const int K = p.K;
-  const long long V = p.V;
-  const SeqInfo *si = p.seq + b;
-  const int n = __ldcg(&si->n);
-  if (n < 0) return;  // invalid sequence: its outputs are written (the same n for all warps)
-  const bool bonus = (n == K);
-  const double St = __ldcg(&si->St), Sd = bonus ? 1.0 : __ldcg(&si->Sd);
-  const float Mt = __ldcg(&si->Mt), Md = bonus ? 0.f : __ldcg(&si->Md);
-  const double c64 = kLog2e / (double)__ldg(p.temperature + b);
+  // ---- this CTA's chunk of the drawn row pair ----
   DrawRow d;
-  d.bonus = bonus;
-  d.Mt = Mt;
-  d.Md = Md;
+  d.bonus = (n == K);
+  d.Mt = sM[n];
+  const double St = sS[n];
+  d.Md = d.bonus ? 0.f : sM[K + 1 + n];
+  const double Sd = d.bonus ? 1.0 : sS[K + 1 + n];
   d.c = make_scale(c64);
-  const double lam = bonus ? 0.0 : St / Sd;
+  const double lam = d.bonus ? 0.0 : St / Sd;
   d.lhi = (float)lam;
   d.llo = (float)(lam - (double)d.lhi);
-  const T *pt = static_cast<const T *>(p.target) + ((long long)b * (K + 1) + n) * V;
-  const T *pd = bonus ? pt : static_cast<const T *>(p.draft) + ((long long)b * K + n) * V;
-  const int head = row_head(pt, V);
-  const long long nvec = (V - head) / VEC;
-  const int NS = p.nru * CW;
-  const double *rp = p.rpart + (long long)b * NS;
-  const double ures = (double)__ldg(p.u_resample + b);
-  int32_t *oty = p.out_tokens + (long long)b * (K + 1) + n;
+  const T *pt = target + (b * (K + 1) + n) * V;
+  const T *pd = d.bonus ? pt : draft + (b * K + n) * V;
 
-  // fp64 prefix over the segment sums (contiguous segments per thread)
-  const int cper = (NS + NTC - 1) / NTC;
-  const int c0 = tid * cper < NS ? tid * cper : NS;
-  const int c1 = c0 + cper < NS ? c0 + cper : NS;
-  double my = 0.0;
-  for (int c2 = c0; c2 < c1; ++c2) my += __ldcg(rp + c2);
-  if (tid == 0) {
-    sm.s_seg = INT_MAX;
-    sm.s_y = INT_MAX;
-    sm.s_lastpos = -1;
-    sm.s_base = -1.0;  // < 0 selects the "last positive element" rule
-  }
-  double cexcl, Z;
-  if (!cta_excl_scan(my, cexcl, Z, sm, cph)) return;
-  if (!bonus && !(Z >= ldexp(St, -64))) {
-    // the fp32 weights ran out of range: redo the draw in fp64
-    int y;
-    double Zx;
-    if (!draw_exact64<T>(pt, pd, V, Mt, St, Md, Sd, c64, ures, sm, cph, y, Zx)) return;
-    if (tid == 0) {
-      *oty = y;
-      if (p.dbg_Z) p.dbg_Z[b] = Zx;
+  const int head = row_head(pt, V);
+  const bool vec_ok = row_head(pd, V) == head;
+  const long long nvec = vec_ok ? (V - head) / VEC : 0;
+  // chunk c covers elements [lo_c, hi_c): chunk 0 also takes the head, and the
+  // chunk whose range holds the < VEC tail elements takes those
+  auto chunk_lo = [&](int cidx) -> long long {
+    if (cidx == 0) return 0;
+    const long long v = head + (long long)cidx * CH;
+    return v < V ? v : V;
+  };
+  auto chunk_hi = [&](int cidx) -> long long {
+    if (cidx == nsr - 1) return V;
+    const long long v = head + (long long)(cidx + 1) * CH;
+    return v < V ? v : V;
+  };
+
+  // Chunk sums: the warps of this CTA take its chunks round robin; a chunk is
+  // 32 lanes x UW vectors of the row pair, summed per lane in fp32 and across
+  // the warp in fp64 with shuffles (no CTA barrier).  Then one arrival ticket.
+  const uint4 *vt = reinterpret_cast<const uint4 *>(pt + head);
+  const uint4 *vd = reinterpret_cast<const uint4 *>(pd + head);
+  const long long tail_chunk = nvec / CHV < nsr - 1 ? nvec / CHV : (long long)(nsr - 1);
+  const int c_beg = cb * cpb;
+  const int c_end = (cb + 1) * cpb < nsr ? (cb + 1) * cpb : nsr;
+  bool wrote = false;
+  for (int chunk = c_beg + warp; chunk < c_end; chunk += NWARP) {
+    float rs = 0.f;
+    if (vec_ok) {
+      uint4 at[UW], ad[UW];
+#pragma unroll
+      for (int k = 0; k < UW; ++k) {
+        const long long vi = (long long)chunk * CHV + (long long)k * 32 + lane;
+        at[k] = vi < nvec ? __ldg(vt + vi) : make_uint4(0, 0, 0, 0);
+        ad[k] = (vi < nvec && !d.bonus) ? __ldg(vd + vi) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int k = 0; k < UW; ++k) {
+        const long long vi = (long long)chunk * CHV + (long long)k * 32 + lane;
+        if (vi < nvec) {
+          float xt[VEC], xd[VEC];
+          Dt<T>::unpack(at[k], xt);
+          Dt<T>::unpack(ad[k], xd);
+#pragma unroll
+          for (int q = 0; q < VEC; ++q) rs += res_weight(xt[q], xd[q], d);
+        }
+      }
+      // head elements (chunk 0) and the < VEC tail elements (their chunk)
+      const long long tail = head + nvec * VEC + lane;
+      const long long extra[2] = {(chunk == 0 && lane < head) ? (long long)lane : -1,
+                                  (chunk == tail_chunk && tail < V && lane < VEC) ? tail : -1};
+#pragma unroll
+      for (int e = 0; e < 2; ++e)
+        if (extra[e] >= 0)
+          rs += res_weight(Dt<T>::load(pt + extra[e]), d.bonus ? 0.f : Dt<T>::load(pd + extra[e]),
+                           d);
+    } else {  // rows of different alignment: scalar loads over the chunk
+      const long long lo = chunk_lo(chunk), hi = chunk_hi(chunk);
+      for (long long v = lo + lane; v < hi; v += 32)
+        rs += res_weight(Dt<T>::load(pt + v), d.bonus ? 0.f : Dt<T>::load(pd + v), d);
     }
-    csync(sm, cph);
+    const double tot = warp_sum((double)rs);
+    if (lane == 0) {
+      ResPartial o;
+      o.R = tot;
+      o.pad = 0.0;
+      rpart[b * nsr + chunk] = o;
+      wrote = true;
+    }
+  }
+  if (wrote) __threadfence();  // chunk sums visible before this CTA's ticket
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const unsigned t = atomicAdd(&counters[b], 1u);
+    s_last = (t == (unsigned)(ncb - 1));
+    s_chunk = INT_MAX;
+    s_y = INT_MAX;
+    s_lastpos = -1;
+  }
+  __syncthreads();
+  if (!s_last) return;
+
+  // ---- the last CTA of sequence b draws ----
+  __threadfence();
+  const ResPartial *rp = rpart + b * nsr;
+  const int cper = (nsr + NT - 1) / NT;  // chunks per thread, contiguous
+  const int c0 = threadIdx.x * cper < nsr ? threadIdx.x * cper : nsr;
+  const int c1 = c0 + cper < nsr ? c0 + cper : nsr;
+  double my = 0.0;
+  for (int c2 = c0; c2 < c1; ++c2) my += __ldcg(&rp[c2].R);
+  double Z;
+  const double cexcl = block_excl_scan(my, Z);
+  if (threadIdx.x == 0) s_mode = (!d.bonus && !(Z >= ldexp(St, -64))) ? 1 : 0;
+  __syncthreads();
+  if (s_mode == 1) {
+    const int y = draw_exact64(pt, pd, V, d.Mt, St, d.Md, Sd, c64, (double)ures, &s_y, &s_lastpos,
+                               dbg_Z ? dbg_Z + b : nullptr);
+    if (threadIdx.x == 0) out_tokens[b * (K + 1) + n] = y;
     return;
   }
-  const double t = ures * Z;
+  const double t = (double)ures * Z;
   {
     double C = cexcl;
     for (int c2 = c0; c2 < c1; ++c2) {
-      const double v = __ldcg(rp + c2);
+      const double v = __ldcg(&rp[c2].R);
       if (C <= t && t < C + v) {
-        atomicMin(&sm.s_seg, c2);
+        atomicMin(&s_chunk, c2);
         break;
       }
       C += v;
     }
   }
-  if (!csync(sm, cph)) return;
-  if (tid == 0) {
-    if (sm.s_seg == INT_MAX) {  // rounding left t at or past the total
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    s_t = t;
+    s_base = -1.0;  // < 0 selects the "last positive element" rule
+    if (s_chunk == INT_MAX) {  // rounding left t at or past the total
       int cs = 0;
-      for (int c2 = NS - 1; c2 >= 0; --c2)
-        if (__ldcg(rp + c2) > 0.0) {
+      for (int c2 = nsr - 1; c2 >= 0; --c2)
+        if (__ldcg(&rp[c2].R) > 0.0) {
           cs = c2;
           break;
         }
-      sm.s_seg = cs;
+      s_chunk = cs;
     }
-    if (p.dbg_Z) p.dbg_Z[b] = Z / St;
+    if (dbg_Z) dbg_Z[b] = Z / St;
   }
-  if (!csync(sm, cph)) return;
-  const int s = sm.s_seg;
-  // the owner of the chosen segment publishes its exclusive prefix
-  if (s >= c0 && s < c1) {
+  __syncthreads();
+  // the owner of the chosen chunk publishes its exclusive prefix
+  if (s_chunk >= c0 && s_chunk < c1) {
     double C = cexcl;
-    for (int c2 = c0; c2 < s; ++c2) C += __ldcg(rp + c2);
-    const double v = __ldcg(rp + s);
-    if (C <= t && t < C + v) sm.s_base = C;
+    for (int c2 = c0; c2 < s_chunk; ++c2) C += __ldcg(&rp[c2].R);
+    const double v = __ldcg(&rp[s_chunk].R);
+    if (C <= t && t < C + v) s_base = C;
   }
-  if (!csync(sm, cph)) return;
+  __syncthreads();
 
-  // rescan of the chosen segment: contiguous elements per thread, in registers
-  long long lo, hi;
-  segment_range<VEC>(s, NS, head, nvec, V, lo, hi);
+  // rescan of the chosen chunk: contiguous elements per thread, in registers
+  const long long lo = chunk_lo(s_chunk), hi = chunk_hi(s_chunk);
   const long long L = hi - lo;
-  const long long E = (L + NTC - 1) / NTC;
-  const long long e0 = lo + (long long)tid * E < hi ? lo + (long long)tid * E : hi;
+  const long long E = (L + NT - 1) / NT;
+  const long long e0 = lo + (long long)threadIdx.x * E < hi ? lo + (long long)threadIdx.x * E : hi;
   const long long e1 = (e0 + E < hi) ? e0 + E : hi;
   float w[EMAX];
 #pragma unroll
   for (int k = 0; k < EMAX; ++k) {
     const long long v = e0 + k;
-    w[k] = (v < e1) ? res_weight(Dt<T>::load(pt + v), bonus ? 0.f : Dt<T>::load(pd + v), d)
+    w[k] = (v < e1) ? res_weight(Dt<T>::load(pt + v), d.bonus ? 0.f : Dt<T>::load(pd + v), d)
                     : 0.0f;
   }
   double mysum = 0.0;
@@ -877,405 +991,35 @@ __device__ __noinline__ void draw_task(const Params &p, int b, Smem &sm, unsigne
     mysum += (double)w[k];
     if (w[k] > 0.0f) lastpos = (int)(e0 + k);
   }
-  double excl, ctot;
-  if (!cta_excl_scan(mysum, excl, ctot, sm, cph)) return;
-  if (lastpos >= 0) atomicMax(&sm.s_lastpos, lastpos);
-  const double base = sm.s_base;
-  if (base >= 0.0) {
-    double C = base + excl;
+  double ctot;
+  const double excl = block_excl_scan(mysum, ctot);
+  if (lastpos >= 0) atomicMax(&s_lastpos, lastpos);
+  if (s_base >= 0.0) {
+    double C = s_base + excl;
 #pragma unroll
     for (int k = 0; k < EMAX; ++k) {
       if (e0 + k < e1) {
         C += (double)w[k];
         if (C > t) {
-          atomicMin(&sm.s_y, (int)(e0 + k));
+          atomicMin(&s_y, (int)(e0 + k));
           break;
         }
       }
     }
   }
-  if (!csync(sm, cph)) return;
-  if (tid == 0) *oty = (sm.s_y != INT_MAX) ? sm.s_y : (sm.s_lastpos >= 0 ? sm.s_lastpos : (int)lo);
-  csync(sm, cph);  // the shared draw state is free again
-}
-
-// ---- the producer thread: claims units, streams tiles, schedules tasks ----
-template <typename T, int U>
-__device__ __noinline__ void producer(const Params &p, Smem &sm, unsigned char *ring) {
-  constexpr int VEC = Dt<T>::VEC;
-  constexpr long long TV = (long long)NTC * U;  // vectors per tile
-  constexpr unsigned TILE_BYTES = (unsigned)TV * 16u;
-  const T *target = static_cast<const T *>(p.target);
-  const T *draft = static_cast<const T *>(p.draft);
-  const int K = p.K, R = 2 * K + 1;
-  const long long V = p.V, B = p.B;
-  const long long S = (long long)R * p.spr, NR = p.nru;
-  unsigned *cnt = p.ctr + kCtrHead;
-
-  int st = 0;       // ring slot of the next entry
-  unsigned ph = 0;  // its phase parity
-  bool copy_last[NSTAGE];     // the last entry pushed into a slot was a copy ...
-  unsigned copy_par[NSTAGE];  // ... of this phase parity
-  for (int i = 0; i < NSTAGE; ++i) copy_last[i] = false, copy_par[i] = 0;
-  // units pushed and not yet retired (FIFO), with their unit-done barriers
-  int pk[NDONE], pb[NDONE], pslot[NDONE];
-  unsigned ppar[NDONE], duse[NDONE];
-  for (int i = 0; i < NDONE; ++i) duse[i] = 0;
-  int phead = 0, npend = 0, dnext = 0;
-  // tasks waiting for a ring slot (FIFO)
-  int tk[NTASKQ], tb[NTASKQ];
-  int thead = 0, ntask = 0;
-  bool abort = false;
-
-  auto advance = [&]() {
-    if (++st == NSTAGE) {
-      st = 0;
-      ph ^= 1u;
-    }
-  };
-  auto acquire = [&]() -> bool {  // the next ring slot is free (bounded wait)
-    if (abort || *(volatile int *)&sm.abort) {
-      abort = true;
-      return false;
-    }
-    if (!mbar_wait(&sm.empty[st], ph ^ 1u)) {
-      abort = true;
-      return false;
-    }
-    return true;
-  };
-  auto push_tasks = [&]() -> bool {
-    while (ntask > 0) {
-      if (!acquire()) return false;
-      Entry &e = sm.ent[st];
-      e.kind = tk[thead];
-      e.b = tb[thead];
-      mbar_arrive(&sm.full[st]);
-      copy_last[st] = false;
-      advance();
-      thead = (thead + 1) % NTASKQ;
-      --ntask;
-    }
-    return true;
-  };
-  // Retire the units the consumers have finished, oldest first (blocking for
-  // the oldest if asked): one arrival on the sequence's counter each; the unit
-  // that completes a sequence's statistics (residual sums) queues its ACCEPT
-  // (DRAW) task.
-  auto retire = [&](bool block) {
-    while (npend > 0 && !abort) {
-      const int i = phead;
-      bool ok;
-      if (block) {
-        ok = mbar_wait(&sm.done[pslot[i]], ppar[i]);
-        block = false;
-        if (!ok) {
-          abort = true;
-          return;
-        }
-      } else {
-        ok = mbar_test(&sm.done[pslot[i]], ppar[i]);
-      }
-      if (!ok) return;
-      phead = (phead + 1) % NDONE;
-      --npend;
-      const long long b = pb[i];
-      const bool stats = pk[i] == E_STATS;
-      const unsigned need = stats ? (unsigned)S : (unsigned)NR;
-      if (atom_add_acq_rel(cnt + 3 * b + (stats ? 0 : 1), 1u) + 1u == need) {
-        const int q = (thead + ntask) % NTASKQ;
-        tk[q] = stats ? E_ACCEPT : E_DRAW;
-        tb[q] = (int)b;
-        ++ntask;
-      }
-    }
-  };
-  // wait until sequence b is decided, retiring units and pushing tasks meanwhile
-  auto wait_ready = [&](long long b) -> bool {
-    const unsigned *flag = cnt + 3 * b + 2;
-    if (ld_acquire(flag)) return true;
-    const unsigned long long t0 = global_ns();
-    for (;;) {
-      retire(false);
-      if (!push_tasks()) return false;
-      if (ld_acquire(flag)) return true;
-      if (abort || (*(volatile unsigned *)&g_error_flags & SPECDEC_ERR_TIMEOUT)) {
-        abort = true;
-        return false;
-      }
-      if (global_ns() - t0 > kWaitNs) {
-        atomicOr(&g_error_flags, SPECDEC_ERR_TIMEOUT);
-        abort = true;
-        return false;
-      }
-      __nanosleep(128);
-    }
-  };
-
-  for (;;) {
-    retire(false);
-    if (!push_tasks() || abort) break;
-    const unsigned u = atomicAdd(p.ctr, 1u);
-    if (u >= p.n_units) break;
-    const UnitRef un = decode_unit(u, B, S, NR, p.lag);
-    while (npend == NDONE && !abort) {  // a unit-done barrier for this unit
-      retire(true);
-      push_tasks();
-    }
-    if (abort) break;
-    const int ds = dnext;
-    dnext = (dnext + 1) % NDONE;
-    const unsigned dpar = duse[ds] & 1u;
-    ++duse[ds];
-    const long long b = un.b;
-    const Scale c = make_scale(kLog2e / (double)__ldg(p.temperature + b));
-    if (un.kind == E_STATS) {
-      const int j = (int)(un.k / p.spr), seg = (int)(un.k - (long long)j * p.spr);
-      const T *row = j <= K ? target + (b * (K + 1) + j) * V : draft + (b * K + (j - K - 1)) * V;
-      const int head = row_head(row, V);
-      const long long nvec = (V - head) / VEC;
-      const uint4 *pv = reinterpret_cast<const uint4 *>(row + head);
-      const int t0 = seg * p.tps, t1 = (t0 + p.tps < p.tpr) ? t0 + p.tps : p.tpr;
-      for (int t = t0; t < t1; ++t) {
-        if (!acquire()) break;
-        const long long v0 = (long long)t * TV;
-        long long nv = nvec - v0;
-        nv = nv < 0 ? 0 : (nv > TV ? TV : nv);
-        Entry &e = sm.ent[st];
-        e.kind = E_STATS;
-        e.b = (int)b;
-        e.j = j;
-        e.flags = (t == t0 ? F_FIRST : 0) | (t == t1 - 1 ? F_LAST : 0) |
-                  ((t == t0 && seg == 0) ? F_HEAD : 0) | ((t == t1 - 1 && t1 == p.tpr) ? F_TAIL : 0);
-        e.nv = (int)nv;
-        e.done = ds;
-        e.unit = (b * R + j) * p.spr + seg;
-        e.chi = c.hi;
-        e.clo = c.lo;
-        e.thr = 64.0f / c.hi;
-        if (nv > 0) {
-          const unsigned bytes = (unsigned)nv * 16u;
-          mbar_arrive_tx(&sm.full[st], bytes);
-          bulk_load(ring + (size_t)st * TILE_BYTES, pv + v0, bytes, &sm.full[st]);
-          copy_last[st] = true;
-          copy_par[st] = ph;
-        } else {
-          mbar_arrive(&sm.full[st]);
-          copy_last[st] = false;
-        }
-        advance();
-      }
-      if (abort) break;
-    } else {
-      if (!wait_ready(b)) break;
-      const SeqInfo *si = p.seq + b;
-      const int n = __ldcg(&si->n);
-      if (!acquire()) break;
-      Entry &e = sm.ent[st];
-      e.kind = E_RES;
-      e.b = (int)b;
-      e.j = (int)un.k;
-      e.done = ds;
-      e.n = n;
-      e.chi = c.hi;
-      e.clo = c.lo;
-      e.Mt = e.Md = e.lhi = e.llo = 0.f;
-      if (n >= 0) {
-        const bool bonus = (n == K);
-        e.Mt = __ldcg(&si->Mt);
-        e.Md = bonus ? 0.f : __ldcg(&si->Md);
-        const double lam = bonus ? 0.0 : __ldcg(&si->St) / __ldcg(&si->Sd);
-        e.lhi = (float)lam;
-        e.llo = (float)(lam - (double)e.lhi);
-      }
-      mbar_arrive(&sm.full[st]);
-      copy_last[st] = false;
-      advance();
-    }
-    const int q = (phead + npend) % NDONE;
-    pk[q] = un.kind;
-    pb[q] = (int)b;
-    pslot[q] = ds;
-    ppar[q] = dpar;
-    ++npend;
-  }
-  // no more units: retire what is in flight, push the tasks that frees, stop
-  while (npend > 0 && !abort) {
-    retire(true);
-    if (!push_tasks()) break;
-  }
-  if (!abort && push_tasks() && acquire()) {
-    sm.ent[st].kind = E_STOP;
-    mbar_arrive(&sm.full[st]);
-    copy_last[st] = false;
-    advance();
-  }
-  if (abort) {
-    // the CTA must not retire with copies in flight
-    atomicExch(&sm.abort, 1);
-    for (int i = 0; i < NSTAGE; ++i)
-      if (copy_last[i]) mbar_wait(&sm.full[i], copy_par[i]);
-  }
-}
-
-// ---- the consumer warps: run the ring's entries in order ----
-template <typename T, int U>
-__device__ __forceinline__ void consumers(const Params &p, Smem &sm, const unsigned char *ring) {
-  constexpr int VEC = Dt<T>::VEC;
-  constexpr int TV = NTC * U;
-  constexpr unsigned TILE_BYTES = (unsigned)TV * 16u;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int K = p.K;
-  const long long V = p.V;
-  unsigned ph = 0, cph = 0;
-  int st = 0;
-  RunStat q;
-  runstat_init(q);
-  Scale c;
-  c.hi = 1.0f;
-  c.lo = 1e-30f;
-  float thr = 64.0f;
-  for (;;) {
-    if (*(volatile int *)&sm.abort) break;
-    if (!__all_sync(FULL, mbar_wait(&sm.full[st], ph))) {
-      if (lane == 0) atomicExch(&sm.abort, 1);
-      break;
-    }
-    const Entry &e = sm.ent[st];
-    const int kind = e.kind;
-    if (kind == E_STATS) {
-      const int flags = e.flags, nv = e.nv;
-      if (flags & F_FIRST) {
-        runstat_init(q);
-        c.hi = e.chi;
-        c.lo = e.clo;
-        thr = e.thr;
-      }
-      // this warp's contiguous quarter of the tile, lanes on consecutive vectors
-      const uint4 *tile = reinterpret_cast<const uint4 *>(ring + (size_t)st * TILE_BYTES);
-      const int base = warp * 32 * U + lane;
-      uint4 v[U];
-      if (nv == TV) {
-#pragma unroll
-        for (int k = 0; k < U; ++k) v[k] = tile[base + k * 32];
-      } else {
-#pragma unroll
-        for (int k = 0; k < U; ++k) {
-          const int vi = base + k * 32;
-          v[k] = vi < nv ? tile[vi] : Dt<T>::neg_inf();
-        }
-      }
-      const int b = e.b, j = e.j, ds = e.done;
-      const long long unit = e.unit;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.empty[st]);
-#pragma unroll
-      for (int k = 0; k < U; ++k) vec_fold<T>(v[k], q, c, thr);
-      if ((flags & (F_HEAD | F_TAIL)) && warp == 0) {  // the row's scalar head / tail
-        const T *row = j <= K ? static_cast<const T *>(p.target) + ((long long)b * (K + 1) + j) * V
-                              : static_cast<const T *>(p.draft) +
-                                    ((long long)b * K + (j - K - 1)) * V;
-        const int head = row_head(row, V);
-        if ((flags & F_HEAD) && lane < head) elem_fold(Dt<T>::load(row + lane), q, c, thr);
-        if (flags & F_TAIL) {
-          const long long tt = head + ((V - head) / VEC) * VEC + lane;
-          if (lane < VEC && tt < V) elem_fold(Dt<T>::load(row + tt), q, c, thr);
-        }
-      }
-      if (flags & F_LAST) {  // this warp's partial of the unit
-        const float m = q.mt;
-        const float sl = runstat_sum_at_max(q, c);
-        const float mw = warp_max_nan(m);
-        double sw = (m == -INFINITY) ? 0.0 : (double)sl * (double)ex2(scaled(m - mw, c));
-        sw = warp_sum(sw);
-        if (lane == 0) {
-          Partial o;
-          o.s = sw;
-          o.m = mw;
-          o.pad = 0;
-          p.part[unit * CW + warp] = o;
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.done[ds]);
-      }
-    } else {
-      const int b = e.b, j = e.j, ds = e.done, n = e.n;
-      DrawRow d;
-      d.Mt = e.Mt;
-      d.Md = e.Md;
-      d.lhi = e.lhi;
-      d.llo = e.llo;
-      d.c.hi = e.chi;
-      d.c.lo = e.clo;
-      d.bonus = (n == K);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.empty[st]);
-      if (kind == E_STOP) break;
-      if (kind == E_RES) {
-        const double r = residual_sum<T>(p, b, j, n, d);
-        if (lane == 0) p.rpart[((long long)b * p.nru + j) * CW + warp] = r;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.done[ds]);
-      } else if (kind == E_ACCEPT) {
-        accept_task<T>(p, b, sm, cph);
-      } else {
-        draw_task<T>(p, b, sm, cph);
-      }
-    }
-    if (++st == NSTAGE) {
-      st = 0;
-      ph ^= 1u;
-    }
-  }
-}
-
-template <typename T, int U>
-__global__ void __launch_bounds__(NTS, kCtasPerSm) k_verify(const __grid_constant__ Params p) {
-  extern __shared__ __align__(128) unsigned char ring[];  // NSTAGE tiles
-  __shared__ Smem sm;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NSTAGE; ++i) {
-      mbar_init(&sm.full[i], 1);
-      mbar_init(&sm.empty[i], CW);
-    }
-    for (int i = 0; i < NDONE; ++i) mbar_init(&sm.done[i], CW);
-    mbar_init(&sm.cbar, CW);
-    sm.abort = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  __syncthreads();
-  if (warp == CW) {
-    if (lane == 0) producer<T, U>(p, sm, ring);
-    __syncwarp();
-  } else {
-    consumers<T, U>(p, sm, ring);
-  }
-  __syncthreads();
-  // the last CTA to leave clears the counters for the next call (and, if a
-  // wait ran out, invalidates every output of this one)
-  if (threadIdx.x == 0) {
-    __threadfence();
-    sm.last_cta = (atomicAdd(p.ctr + 1, 1u) == gridDim.x - 1) ? 1 : 0;
-  }
-  __syncthreads();
-  if (sm.last_cta) {
-    __threadfence();
-    if (*(volatile unsigned *)&g_error_flags & SPECDEC_ERR_TIMEOUT) {
-      const long long nt = (long long)p.B * (p.K + 1);
-      for (long long i = threadIdx.x; i < nt; i += blockDim.x) p.out_tokens[i] = -1;
-      for (long long i = threadIdx.x; i < p.B; i += blockDim.x) p.out_n[i] = -1;
-    }
-    const long long nw = counter_words(p.B);
-    for (long long i = threadIdx.x; i < nw; i += blockDim.x) p.ctr[i] = 0u;
+    int y = s_y;
+    if (y == INT_MAX) y = (s_lastpos >= 0) ? s_lastpos : (int)lo;
+    out_tokens[b * (K + 1) + n] = y;
   }
 }
 
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-enum KernelId { KID_VERIFY = 0, KID_COUNT = 1 };
-const char *kKernelNames[KID_COUNT] = {"k_verify"};
+enum KernelId { KID_STATS = 0, KID_FINISH = 1, KID_COUNT = 2 };
+const char *kKernelNames[KID_COUNT] = {"k_row_stats", "k_finish"};
 
 std::mutex g_mu;
 uint64_t g_launches[KID_COUNT];
@@ -1294,32 +1038,10 @@ std::unordered_map<int, DeviceBuf> g_staging;  // end-to-end staging per device
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// The counter region of a workspace of W bytes: its first bytes, sized by W
-// alone, so that every call on one workspace finds its counters where the
-// previous calls left them zero, whatever their sizes.  A call on B sequences
-// uses 4 + 3B words of it; every call needs at least 384 B of records per
-// sequence, so a workspace that holds a call's records also holds its
-// counters.
-inline size_t counter_region(size_t W) { return align256(64 + W / 16); }
-// bytes of records a workspace of W bytes holds after its counter region
-inline size_t record_capacity(size_t W) {
-  const size_t c = counter_region(W);
-  return W > c ? W - c : 0;
-}
-
-#ifndef SPECDEC_TILES_PER_UNIT
-#define SPECDEC_TILES_PER_UNIT 0  // 0: chosen from the sizes
-#endif
-#ifndef SPECDEC_LAG_TILES_PER_CTA
-#define SPECDEC_LAG_TILES_PER_CTA 10
-#endif
-
 struct Plan {
-  int esize, vec, U, tpr, tps, spr, nru;
-  long long rows, tiles;
-  unsigned n_units;
-  size_t off_part, off_rpart, off_seq, records;  // inside the record region
-  size_t total;                                  // smallest workspace that holds them
+  int esize, vec, U, tpr, slots, nsr, cpb;
+  long long rows, tiles, G1;  // G1: CTAs of the statistics sweep
+  size_t off_part, off_rpart, off_cnt, total;
 };
 
 int num_sms() {
@@ -1328,20 +1050,19 @@ int num_sms() {
   return n > 0 ? n : 148;
 }
 
+
 // Work decomposition for these sizes; a pure function of the sizes and the SM
 // count, so repeated calls reduce in the same order (bit-reproducible).
 bool make_plan(int B, int K, int V, specdec_dtype dtype, int sms, Plan &pl) {
   if (B < 0 || K < 1 || K > 32 || V < 1) return false;
   if (dtype != SPECDEC_F32 && dtype != SPECDEC_BF16) return false;
-  if ((long long)B * (K + 1) * (long long)V > (1LL << 56)) return false;
   pl.esize = dtype == SPECDEC_BF16 ? 2 : 4;
   pl.vec = 16 / pl.esize;
-  const int R = 2 * K + 1;
-  pl.rows = (long long)B * R;
+  pl.rows = (long long)B * (2 * K + 1);
   const long long nvec_max = ((long long)V + pl.vec - 1) / pl.vec;
-  const long long cap = (long long)kCtasPerSm * sms;
   // tiles of 4 vectors per consumer thread (16 KB); 1 vector per thread when
   // 16 KB tiles would leave SMs idle (single-sequence batches)
+  const long long cap = (long long)kStatsCtasPerSm * sms;
   long long tpr = (nvec_max + NTC * 4 - 1) / (NTC * 4);
   pl.U = 4;
   if (pl.rows * tpr < 2 * cap) {
@@ -1349,30 +1070,31 @@ bool make_plan(int B, int K, int V, specdec_dtype dtype, int sms, Plan &pl) {
     tpr = (nvec_max + NTC - 1) / NTC;
   }
   if (tpr < 1) tpr = 1;
-  if (tpr > INT_MAX / 4) return false;
   pl.tpr = (int)tpr;
   pl.tiles = pl.rows * tpr;
-  int tps = SPECDEC_TILES_PER_UNIT;
-  if (tps <= 0) tps = (pl.tiles >= 16 * cap) ? 2 : 1;
-  if (tps > pl.tpr) tps = pl.tpr;
-  pl.tps = tps;
-  pl.spr = (pl.tpr + tps - 1) / tps;
-  const long long nru = (nvec_max + RV - 1) / RV;
-  pl.nru = (int)(nru > 0 ? nru : 1);
-  const long long units = (long long)B * ((long long)R * pl.spr + pl.nru);
-  if (units >= (1LL << 31)) return false;
-  pl.n_units = (unsigned)units;
+  pl.G1 = pl.tiles < cap ? pl.tiles : cap;
+  // partial slots per row: the most CTAs whose tile ranges meet one row
+  const long long minr = pl.tiles / pl.G1;  // shortest range
+  pl.slots = (int)((tpr - 1 + minr - 1) / minr + 1);
+  // k_finish chunks: 32 lanes x kFinishUW vectors of the drawn row pair
+  const long long nr = (nvec_max + 32LL * kFinishUW - 1) / (32LL * kFinishUW);
+  pl.nsr = (int)(nr > 0 ? nr : 1);
+  // chunks per CTA of k_finish: as many CTAs per sequence as keep the whole
+  // grid inside one wave (each CTA repeats the small acceptance step)
+  long long ncb = (long long)kFinishCtasPerSm * sms / (B > 0 ? B : 1);
+  if (ncb < 1) ncb = 1;
+  if (ncb > pl.nsr) ncb = pl.nsr;
+  pl.cpb = (int)((pl.nsr + ncb - 1) / ncb);
+  if ((long long)B * pl.nsr > INT_MAX) return false;
+  if ((long long)B * (K + 1) * (long long)V > (1LL << 56)) return false;
   size_t off = 0;
   pl.off_part = off;
-  off = align256(off + sizeof(Partial) * (size_t)pl.rows * pl.spr * CW);
+  off = align256(off + sizeof(Partial) * (size_t)pl.rows * pl.slots * CW);
   pl.off_rpart = off;
-  off = align256(off + sizeof(double) * (size_t)B * pl.nru * CW);
-  pl.off_seq = off;
-  off = align256(off + sizeof(SeqInfo) * (size_t)B);
-  pl.records = off;
-  size_t W = align256(off + off / 15 + 512);
-  while (record_capacity(W) < off) W += 256;
-  pl.total = W;
+  off = align256(off + sizeof(ResPartial) * (size_t)B * pl.nsr);
+  pl.off_cnt = off;
+  off = align256(off + sizeof(unsigned) * (size_t)B);
+  pl.total = off > 0 ? off : 256;
   return true;
 }
 
@@ -1392,10 +1114,29 @@ int resident_ctas(KernelT kernel, int threads, size_t smem) {
   if (it != cache.end()) return it->second;
   cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem) != cudaSuccess)
-    n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem) != cudaSuccess ||
+      n < 1)
+    n = 1;
   cache[key] = n;
   return n;
+}
+
+// launch with programmatic stream serialisation: the kernel may be scheduled
+// while the previous one drains and waits for it with cudaGridDependencySynchronize
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, cudaStream_t st,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
 struct LaunchTimer {
@@ -1420,35 +1161,45 @@ struct LaunchTimer {
   }
 };
 
-// One cooperative launch: every CTA is resident for the whole kernel, which
-// the waits between CTAs rely on for progress.
-template <typename T, int U>
-specdec_status launch_verify(Params prm, const Plan &pl, cudaStream_t st) {
-  auto kern = k_verify<T, U>;
-  const size_t smem = (size_t)NSTAGE * NTC * U * 16;
-  const int per_sm = resident_ctas(kern, NTS, smem);
-  if (per_sm < 1) return SPECDEC_ECUDA;
-  const long long cap = (long long)per_sm * num_sms();
-  const unsigned grid = (unsigned)((long long)pl.n_units < cap ? (long long)pl.n_units : cap);
-  // lag of the residual units behind the statistics units, in sequences: about
-  // SPECDEC_LAG_TILES_PER_CTA tiles per CTA of the grid
-  const long long tiles_per_seq = (long long)(2 * prm.K + 1) * pl.tpr;
-  long long lag = ((long long)SPECDEC_LAG_TILES_PER_CTA * grid + tiles_per_seq - 1) / tiles_per_seq;
-  if (lag < 1) lag = 1;
-  if (lag > prm.B) lag = prm.B;
-  prm.lag = (int)lag;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(NTS);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  LaunchTimer lt(KID_VERIFY, st);
-  return cudaLaunchKernelEx(&cfg, kern, prm) == cudaSuccess ? SPECDEC_OK : SPECDEC_ECUDA;
+template <typename T>
+specdec_status launch_all(const void *tg, const void *dr, const int32_t *tok, const float *ua,
+                          const float *ur, const float *temp, int B, int K, int V,
+                          const Plan &pl, char *ws, const specdec_debug *dbg, int32_t *out_tokens,
+                          int32_t *out_n, cudaStream_t st) {
+  const T *t = static_cast<const T *>(tg);
+  const T *d = static_cast<const T *>(dr);
+  Partial *part = reinterpret_cast<Partial *>(ws + pl.off_part);
+  ResPartial *rp = reinterpret_cast<ResPartial *>(ws + pl.off_rpart);
+  unsigned *cnt = reinterpret_cast<unsigned *>(ws + pl.off_cnt);
+  StatsGeom g;
+  g.K = K;
+  g.V = V;
+  g.tpr = pl.tpr;
+  g.tiles = pl.tiles;
+  g.slots = pl.slots;
+  cudaError_t e = cudaSuccess;
+  {
+    LaunchTimer lt(KID_STATS, st);
+    auto kern = pl.U == 4 ? k_row_stats<T, 4> : k_row_stats<T, 1>;
+    const size_t smem = (size_t)NSTAGE * NTC * pl.U * 16;
+    // the sweep assumes its CTAs are co-resident only for speed, not for
+    // progress: nothing waits on another CTA
+    resident_ctas(kern, NTS, smem);
+    kern<<<(unsigned)pl.G1, NTS, smem, st>>>(t, d, temp, g, part, cnt, B);
+    e = cudaGetLastError();
+  }
+  if (e != cudaSuccess) return SPECDEC_ECUDA;
+  {
+    LaunchTimer lt(KID_FINISH, st);
+    const unsigned g2 = (unsigned)((long long)B * ((pl.nsr + pl.cpb - 1) / pl.cpb));
+    auto kern = k_finish<T, kFinishUW>;
+    e = launch_pdl(kern, g2, NT, st, t, d, tok, ua, ur, temp, K, (long long)V, pl.tpr, pl.tiles,
+                   pl.G1, pl.slots, pl.nsr, pl.cpb,
+                   (const Partial *)part, rp, cnt, out_tokens, out_n,
+                   dbg ? dbg->row_max : nullptr, dbg ? dbg->row_sum : nullptr,
+                   dbg ? dbg->p_x : nullptr, dbg ? dbg->q_x : nullptr, dbg ? dbg->Z : nullptr);
+  }
+  return e == cudaSuccess ? SPECDEC_OK : SPECDEC_ECUDA;
 }
 
 specdec_status check_args(const void *tg, const void *dr, const int32_t *tok, const float *ua,
@@ -1468,8 +1219,6 @@ specdec_status check_args(const void *tg, const void *dr, const int32_t *tok, co
   return SPECDEC_OK;
 }
 
-// ws / ws_bytes: a workspace whose counter region (counter_region(ws_bytes)
-// first bytes) is zero, as every call leaves it
 specdec_status run(const void *tg, const void *dr, const int32_t *tok, const float *ua,
                    const float *ur, const float *temp, int B, int K, int V, specdec_dtype dtype,
                    void *ws, size_t ws_bytes, const specdec_debug *dbg, int32_t *ot, int32_t *on,
@@ -1478,45 +1227,17 @@ specdec_status run(const void *tg, const void *dr, const int32_t *tok, const flo
   if (s != SPECDEC_OK || B == 0) return s;
   Plan pl;
   if (!make_plan(B, K, V, dtype, num_sms(), pl)) return SPECDEC_EINVAL;
-  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255) || record_capacity(ws_bytes) < pl.records)
-    return SPECDEC_EINVAL;
-  char *rec = static_cast<char *>(ws) + counter_region(ws_bytes);
-  Params prm;
-  prm.target = tg;
-  prm.draft = dr;
-  prm.tokens = tok;
-  prm.u_accept = ua;
-  prm.u_resample = ur;
-  prm.temperature = temp;
-  prm.B = B;
-  prm.K = K;
-  prm.V = V;
-  prm.tpr = pl.tpr;
-  prm.tps = pl.tps;
-  prm.spr = pl.spr;
-  prm.nru = pl.nru;
-  prm.lag = 1;
-  prm.n_units = pl.n_units;
-  prm.part = reinterpret_cast<Partial *>(rec + pl.off_part);
-  prm.rpart = reinterpret_cast<double *>(rec + pl.off_rpart);
-  prm.seq = reinterpret_cast<SeqInfo *>(rec + pl.off_seq);
-  prm.ctr = static_cast<unsigned *>(ws);
-  prm.out_tokens = ot;
-  prm.out_n = on;
-  prm.dbg_row_max = dbg ? dbg->row_max : nullptr;
-  prm.dbg_row_sum = dbg ? dbg->row_sum : nullptr;
-  prm.dbg_px = dbg ? dbg->p_x : nullptr;
-  prm.dbg_qx = dbg ? dbg->q_x : nullptr;
-  prm.dbg_Z = dbg ? dbg->Z : nullptr;
+  if (!ws || ws_bytes < pl.total || (reinterpret_cast<uintptr_t>(ws) & 255)) return SPECDEC_EINVAL;
   if (dtype == SPECDEC_BF16)
-    return pl.U == 4 ? launch_verify<__nv_bfloat16, 4>(prm, pl, st)
-                     : launch_verify<__nv_bfloat16, 1>(prm, pl, st);
-  return pl.U == 4 ? launch_verify<float, 4>(prm, pl, st) : launch_verify<float, 1>(prm, pl, st);
+    return launch_all<__nv_bfloat16>(tg, dr, tok, ua, ur, temp, B, K, V, pl,
+                                     static_cast<char *>(ws), dbg, ot, on, st);
+  return launch_all<float>(tg, dr, tok, ua, ur, temp, B, K, V, pl, static_cast<char *>(ws), dbg,
+                           ot, on, st);
 }
 
 // grow-only device buffer of the current device (zero-filled when (re)allocated)
 specdec_status ensure_buf(std::unordered_map<int, DeviceBuf> &map, size_t bytes,
-                          cudaStream_t st, void **out, size_t *out_bytes) {
+                          cudaStream_t st, void **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SPECDEC_ECUDA;
   std::lock_guard<std::mutex> lk(g_mu);
@@ -1541,12 +1262,10 @@ specdec_status ensure_buf(std::unordered_map<int, DeviceBuf> &map, size_t bytes,
     db.bytes = bytes;
   }
   *out = db.ptr;
-  if (out_bytes) *out_bytes = db.bytes;
   return SPECDEC_OK;
 }
 
 }  // namespace
-
 
 // ---------------------------------------------------------------------------
 // Fixed scratch for specdec_verify_static.  Some callers cannot allocate device
@@ -1593,16 +1312,6 @@ size_t specdec_workspace_bytes(int B, int K, int V, specdec_dtype dtype) {
   return pl.total;
 }
 
-specdec_status specdec_workspace_init(void *workspace, size_t workspace_bytes, void *stream) {
-  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255) || workspace_bytes < 256)
-    return SPECDEC_EINVAL;
-  size_t n = counter_region(workspace_bytes);
-  if (n > workspace_bytes) n = workspace_bytes;
-  return cudaMemsetAsync(workspace, 0, n, static_cast<cudaStream_t>(stream)) == cudaSuccess
-             ? SPECDEC_OK
-             : SPECDEC_ECUDA;
-}
-
 specdec_status specdec_verify_ex(const void *target_logits, const void *draft_logits,
                                  const int32_t *draft_tokens, const float *u_accept,
                                  const float *u_resample, const float *temperature, int B,
@@ -1625,11 +1334,10 @@ specdec_status specdec_verify(const void *target_logits, const void *draft_logit
   const size_t need = specdec_workspace_bytes(B, K, V, dtype);
   if (need == 0) return SPECDEC_EINVAL;
   void *ws = nullptr;
-  size_t ws_bytes = 0;
-  s = ensure_buf(g_ws, need, static_cast<cudaStream_t>(stream), &ws, &ws_bytes);
+  s = ensure_buf(g_ws, need, static_cast<cudaStream_t>(stream), &ws);
   if (s != SPECDEC_OK) return s;
   return run(target_logits, draft_logits, draft_tokens, u_accept, u_resample, temperature, B, K,
-             V, dtype, ws, ws_bytes, nullptr, out_tokens, out_num_accepted,
+             V, dtype, ws, need, nullptr, out_tokens, out_num_accepted,
              static_cast<cudaStream_t>(stream));
 }
 
@@ -1666,17 +1374,16 @@ specdec_status specdec_verify_host(const void *target_logits, const void *draft_
   const size_t n_t = (size_t)B * (K + 1) * (size_t)V * es, n_d = (size_t)B * K * (size_t)V * es;
   const size_t n_tok = sizeof(int32_t) * (size_t)B * K, n_ua = sizeof(float) * (size_t)B * K;
   const size_t n_b = sizeof(float) * (size_t)B, n_ot = sizeof(int32_t) * (size_t)B * (K + 1);
-  size_t off[8], tot = 0;
+  size_t off[9], tot = 0;
   const size_t sizes[8] = {n_t, n_d, n_tok, n_ua, n_b, n_b, n_ot, n_b};
   for (int i = 0; i < 8; ++i) {
     off[i] = tot;
     tot = align256(tot + sizes[i]);
   }
-  void *base = nullptr, *ws = nullptr;
-  size_t ws_bytes = 0;
-  s = ensure_buf(g_staging, tot, st, &base, nullptr);
-  if (s != SPECDEC_OK) return s;
-  s = ensure_buf(g_ws, pl.total, st, &ws, &ws_bytes);
+  off[8] = tot;
+  tot += pl.total;
+  void *base = nullptr;
+  s = ensure_buf(g_staging, tot, st, &base);
   if (s != SPECDEC_OK) return s;
   char *c = static_cast<char *>(base);
   const void *src[6] = {target_logits, draft_logits, draft_tokens, u_accept, u_resample,
@@ -1686,7 +1393,8 @@ specdec_status specdec_verify_host(const void *target_logits, const void *draft_
       return SPECDEC_ECUDA;
   s = run(c + off[0], c + off[1], reinterpret_cast<const int32_t *>(c + off[2]),
           reinterpret_cast<const float *>(c + off[3]), reinterpret_cast<const float *>(c + off[4]),
-          reinterpret_cast<const float *>(c + off[5]), B, K, V, dtype, ws, ws_bytes, nullptr, reinterpret_cast<int32_t *>(c + off[6]), reinterpret_cast<int32_t *>(c + off[7]),
+          reinterpret_cast<const float *>(c + off[5]), B, K, V, dtype, c + off[8], pl.total,
+          nullptr, reinterpret_cast<int32_t *>(c + off[6]), reinterpret_cast<int32_t *>(c + off[7]),
           st);
   if (s != SPECDEC_OK) return s;
   if (cudaMemcpyAsync(out_tokens, c + off[6], n_ot, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
@@ -1714,15 +1422,15 @@ specdec_status specdec_verify_static(const void *target_logits, const void *draf
   specdec_status s = check_args(target_logits, draft_logits, draft_tokens, u_accept, u_resample,
                                 temperature, B, K, V, dtype, out_tokens, out_num_accepted);
   if (s != SPECDEC_OK || B == 0) return s;
-  Plan pl;
-  if (!make_plan(B, K, V, dtype, num_sms(), pl)) return SPECDEC_EINVAL;
-  if (record_capacity((size_t)SPECDEC_STATIC_SCRATCH_BYTES) < pl.records) return SPECDEC_ESIZE;
+  const size_t need = specdec_workspace_bytes(B, K, V, dtype);
+  if (need == 0) return SPECDEC_EINVAL;
+  if (need > (size_t)SPECDEC_STATIC_SCRATCH_BYTES) return SPECDEC_ESIZE;
   void *scratch = nullptr;
   s = static_scratch_address(&scratch);
   if (s != SPECDEC_OK) return s;
-  // The array starts zeroed (it is a zero-initialised device variable) and
-  // every call leaves its counter region zeroed again; the records the kernel
-  // reads are written earlier in the same call.
+  // Nothing in the scratch has to start at zero: every record the kernels read
+  // (V-split partials, per-sequence selection, chunk sums, the arrival counters
+  // that k_accept resets) is written earlier in the same call.
   return run(target_logits, draft_logits, draft_tokens, u_accept, u_resample, temperature, B, K,
              V, dtype, scratch, (size_t)SPECDEC_STATIC_SCRATCH_BYTES, nullptr, out_tokens,
              out_num_accepted, static_cast<cudaStream_t>(stream));

@@ -60,9 +60,7 @@ def gpu_verify(x, debug=True, dev_inputs=None, garbage_workspace=False):
         if garbage_workspace:
             dt = sd.SPECDEC_BF16 if x.dtype == "bf16" else sd.SPECDEC_F32
             n = sd.specdec_workspace_bytes(B, K, x.V, dt)
-            # garbage everywhere but the counter region, which workspace_init zeroes
             ws = torch.randint(0, 255, (n,), dtype=torch.uint8, device=dev)
-            sd.workspace_init(ws)
         ot, on = sd.verify(d["target"], d["draft"], d["tokens"], d["u_accept"], d["u_resample"],
                            d["temperature"], debug=dbg, workspace=ws)
         torch.cuda.synchronize()
