@@ -54,6 +54,8 @@ def parse():
                     help="minimum oracle time for the cpu_baseline leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-timing", choices=["on", "off"], default="on")
+    ap.add_argument("--early-exit", choices=["on", "off"], default="on",
+                    help="also time specdec_verify_early_exit on the same steps")
     return ap.parse_args()
 
 
@@ -319,6 +321,37 @@ def run_cuda(args):
     total_bytes = floor * world
     gbs = total_bytes / (ms_step * 1e-3) / 1e9
 
+    # ---- early exit: the same steps through specdec_verify_early_exit -------
+    early = None
+    if args.early_exit == "on":
+        fe = L.specdec_verify_early_exit
+        for i in range(3):
+            if fe(*calls[i % ncopies]) != 0:
+                raise RuntimeError("specdec_verify_early_exit failed")
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for i in range(args.steps):
+            fe(*calls[i % ncopies])
+        f1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms_ee = sdist.max_over_ranks(f0.elapsed_time(f1), dev) / args.steps
+        n_ee = bufs[0]["on"].cpu().numpy()
+        same_tokens = bool(np.array_equal(bufs[0]["ot"].cpu().numpy(), ref_tok.numpy()))
+        P = 2 if K >= 2 else K
+        rows_read = int(np.sum(np.where(n_ee >= P, 2 * K + 1, 2 * P)))
+        read_bytes = rows_read * V * (2 if w.dtype == "bf16" else 4)
+        early = {"ms_per_step": ms_ee, "value": total_bytes / (ms_ee * 1e-3) / 1e9, "unit": "GB/s",
+                 "rows_read_fraction": rows_read / (B * (2 * K + 1)),
+                 "read_GBs": read_bytes * world / (ms_ee * 1e-3) / 1e9,
+                 "tokens_equal_full_call": same_tokens,
+                 "note": "value counts the full two-tensor floor per step, as the headline "
+                         "does; read_GBs counts the rows this call actually reads"}
+
     # ---- end to end through the host entry point (pinned buffers) ----------
     pin = {k: torch.from_numpy(np.ascontiguousarray(getattr(x, k))).pin_memory()
            for k in ("target", "draft", "tokens", "u_accept", "u_resample", "temperature")}
@@ -381,6 +414,8 @@ def run_cuda(args):
                             "timing": "CUDA events around each launch on its stream, over a "
                                       "second run of the K steps"}
         line["kernel_us"] = {k: (v[0] / max(v[1], 1) * 1e3) for k, v in kern.items()}
+    if early is not None:
+        line["early_exit"] = early
     line["e2e"] = {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                    "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
     line["clocks"] = sampler.summary()

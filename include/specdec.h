@@ -139,6 +139,41 @@ specdec_status specdec_verify_ex(const void *target_logits, const void *draft_lo
                                  size_t workspace_bytes, const specdec_debug *dbg,
                                  int32_t *out_tokens, int32_t *out_num_accepted, void *stream);
 
+/* Early-exit verify: the same operation, the same outputs, fewer bytes read.
+ *
+ * The pages stop the verification at the first rejected draft token (the
+ * speculative decoding blog, "The mathematical definition from Leviathan et
+ * al.": tokens are checked in order and the first disagreement ends the step;
+ * the SMC-SD page, section 1 and "Key differences from standard SD": in
+ * standard SD the first rejection truncates the draft block and the tokens
+ * after it are discarded).  The rows of positions after the first
+ * rejection (and the target's bonus row unless every draft token is accepted)
+ * never influence the result, so they need not be read.  This call reads the
+ * rows of positions 0 and 1 of every sequence first, decides the sequences
+ * rejected there, and then reads positions 2..K-1 and the bonus row only of the
+ * sequences that accepted both: two statistics sweeps and two finish passes
+ * instead of one of each.  Worth it when acceptance is low (at mean acceptance
+ * a it reads about (4 + a^2 (2K-3)) / (2K+1) of the logits); at high acceptance
+ * the second pass costs more launch latency than it saves.
+ * Arguments, layouts, errors and results are those of specdec_verify /
+ * specdec_verify_ex (diagnostics: row statistics only of the rows read, p_x
+ * and q_x of the positions tested).  The row statistics are reduced over a
+ * different split of the rows than in specdec_verify, so probabilities agree
+ * with it to rounding (a few 1e-7) rather than bit for bit. */
+specdec_status specdec_verify_early_exit(const void *target_logits, const void *draft_logits,
+                                         const int32_t *draft_tokens, const float *u_accept,
+                                         const float *u_resample, const float *temperature,
+                                         int B, int K, int V, specdec_dtype dtype,
+                                         int32_t *out_tokens, int32_t *out_num_accepted,
+                                         void *stream);
+specdec_status specdec_verify_early_exit_ex(const void *target_logits, const void *draft_logits,
+                                            const int32_t *draft_tokens, const float *u_accept,
+                                            const float *u_resample, const float *temperature,
+                                            int B, int K, int V, specdec_dtype dtype,
+                                            void *workspace, size_t workspace_bytes,
+                                            const specdec_debug *dbg, int32_t *out_tokens,
+                                            int32_t *out_num_accepted, void *stream);
+
 /* End-to-end variant: every pointer is HOST memory (pinned memory makes the
  * copies asynchronous).  Copies the inputs to library-owned device buffers,
  * runs the verify step on `stream`, copies the outputs back and synchronises

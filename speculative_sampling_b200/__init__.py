@@ -32,6 +32,9 @@ _SIGS = {
     "specdec_verify_ex": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, ctypes.c_size_t, _P,
                                _P, _P, _P]),
     "specdec_verify_host": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P]),
+    "specdec_verify_early_exit": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P]),
+    "specdec_verify_early_exit_ex": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P,
+                                          ctypes.c_size_t, _P, _P, _P, _P]),
     "specdec_verify_static": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P]),
     "specdec_device_errors": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
     "specdec_release": (None, []),
@@ -115,6 +118,22 @@ def specdec_verify_ex(target, draft, tokens, u_accept, u_resample, temperature, 
                                    out_num_accepted, stream)
 
 
+def specdec_verify_early_exit(target, draft, tokens, u_accept, u_resample, temperature, B, K,
+                              V, dtype, out_tokens, out_num_accepted, stream) -> int:
+    return lib().specdec_verify_early_exit(target, draft, tokens, u_accept, u_resample,
+                                           temperature, B, K, V, dtype, out_tokens,
+                                           out_num_accepted, stream)
+
+
+def specdec_verify_early_exit_ex(target, draft, tokens, u_accept, u_resample, temperature, B, K,
+                                 V, dtype, workspace, workspace_bytes, dbg, out_tokens,
+                                 out_num_accepted, stream) -> int:
+    return lib().specdec_verify_early_exit_ex(target, draft, tokens, u_accept, u_resample,
+                                              temperature, B, K, V, dtype, workspace,
+                                              workspace_bytes, dbg, out_tokens,
+                                              out_num_accepted, stream)
+
+
 def specdec_verify_host(target, draft, tokens, u_accept, u_resample, temperature, B, K, V,
                         dtype, out_tokens, out_num_accepted, stream) -> int:
     return lib().specdec_verify_host(target, draft, tokens, u_accept, u_resample, temperature,
@@ -182,7 +201,8 @@ def _check_dev(*ts):
 
 
 def verify(target, draft, tokens, u_accept, u_resample, temperature, out_tokens=None,
-           out_num_accepted=None, stream=None, workspace=None, debug: Optional[dict] = None):
+           out_num_accepted=None, stream=None, workspace=None, debug: Optional[dict] = None,
+           early_exit: bool = False):
     """Run the verify step on CUDA tensors.
 
     target [B,K+1,V] and draft [B,K,V] (bfloat16 or float32), tokens [B,K]
@@ -191,7 +211,8 @@ def verify(target, draft, tokens, u_accept, u_resample, temperature, out_tokens=
     asynchronously on ``stream`` (default: torch's current stream).  With
     ``workspace`` (a uint8 CUDA tensor of specdec_workspace_bytes bytes) or
     ``debug`` (dict of preallocated tensors named as specdec_debug's fields)
-    the call goes through specdec_verify_ex."""
+    the call goes through specdec_verify_ex.  ``early_exit`` selects the
+    early-exit entry points (same results, fewer rows read)."""
     import torch
     B, K1, V = target.shape
     K = K1 - 1
@@ -214,8 +235,10 @@ def verify(target, draft, tokens, u_accept, u_resample, temperature, out_tokens=
     args = (target.data_ptr(), draft.data_ptr(), tokens.data_ptr(), u_accept.data_ptr(),
             u_resample.data_ptr(), temperature.data_ptr(), B, K, V, dt)
     if workspace is None and debug is None:
-        st = specdec_verify(*args, out_tokens.data_ptr(), out_num_accepted.data_ptr(), stream)
-        _chk(st, "specdec_verify")
+        f, name = ((specdec_verify_early_exit, "specdec_verify_early_exit") if early_exit
+                   else (specdec_verify, "specdec_verify"))
+        st = f(*args, out_tokens.data_ptr(), out_num_accepted.data_ptr(), stream)
+        _chk(st, name)
         return out_tokens, out_num_accepted
     need = specdec_workspace_bytes(B, K, V, dt)
     if workspace is None:
@@ -227,9 +250,11 @@ def verify(target, draft, tokens, u_accept, u_resample, temperature, out_tokens=
             t = debug.get(f)
             setattr(d, f, t.data_ptr() if t is not None else None)
         dbg = ctypes.byref(d)
-    st = specdec_verify_ex(*args, workspace.data_ptr(), workspace.numel(), dbg,
-                           out_tokens.data_ptr(), out_num_accepted.data_ptr(), stream)
-    _chk(st, "specdec_verify_ex")
+    f, name = ((specdec_verify_early_exit_ex, "specdec_verify_early_exit_ex") if early_exit
+               else (specdec_verify_ex, "specdec_verify_ex"))
+    st = f(*args, workspace.data_ptr(), workspace.numel(), dbg, out_tokens.data_ptr(),
+           out_num_accepted.data_ptr(), stream)
+    _chk(st, name)
     return out_tokens, out_num_accepted
 
 

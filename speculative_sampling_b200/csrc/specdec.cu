@@ -62,6 +62,10 @@ struct __align__(16) Partial {  // one (row, V-split): max and sum of 2^((z-m)c)
   float m;
   uint32_t pad;
 };
+struct __align__(16) SeqInfo {  // a sequence decided by an earlier pass (early exit)
+  double St, Sd;                // row sums (at the row max) of the drawn pair
+  float Mt, Md;                 // row maxima of the drawn pair
+};
 struct __align__(16) ResPartial {  // one (sequence, V-chunk) of the drawn row(s)
   double R;                        // sum of St * max(0, p - q)  (or of 2^((z-m)c), bonus)
   double pad;
@@ -350,13 +354,24 @@ __device__ __forceinline__ void elem_fold(float x, RunStat &q, Scale c, float th
   q.acc.x += ex2(scaled(x + q.nr, c));
 }
 
+// A sweep covers a window of draft positions [p0, p0 + np) (both the target
+// and the draft row of each) and, when `bonus` is set, the target's row K.
+// Within a sequence the window's rows are walked as target p0, draft p0,
+// target p0+1, ..., then the bonus row: rps rows per sequence.  With `state`
+// set, only the sequences still undecided (state[b] == kSeqActive) are read.
+constexpr int kSeqActive = -2;
 struct StatsGeom {
   int K;
   long long V;
   int tpr;          // tiles per row
   long long tiles;  // rows * tpr
   int slots;        // CTA slots per row (>= CTAs that can share one row)
+  int p0, np, rps;  // the window: first position, positions, rows per sequence
+  const int *state; // per-sequence decision state, or null (every sequence)
 };
+__device__ __forceinline__ bool seq_active(const StatsGeom &g, long long b) {
+  return g.state == nullptr || __ldcg(g.state + b) == kSeqActive;
+}
 
 // CTA g of G owns tiles [g*T/G, (g+1)*T/G); the owner of tile t is then
 // floor(((t+1)*G - 1) / T).  Both the statistics kernel and the combine in
@@ -369,37 +384,37 @@ __host__ __device__ __forceinline__ long long tile_owner(long long t, long long 
   return ((t + 1) * G - 1) / T;
 }
 
-// The current row of a CTA's tile walk.  Rows are numbered b*(2K+1) + j with
-// j = 0..K the target rows and j = K+1..2K the draft rows of sequence b; the
-// cursor steps row by row without divisions.
+// The current row of a CTA's tile walk.  Rows are numbered b*rps + w, w the
+// row of the window (see StatsGeom); the cursor steps row by row without
+// divisions.
 template <typename T>
 struct RowCursor {
   const T *p;
   const uint4 *pv;
   long long row, b, nvec;
-  int j, ti, head;
+  int w, ti, head;
   __device__ __forceinline__ void point(const T *target, const T *draft, const StatsGeom &g) {
     constexpr int VEC = Dt<T>::VEC;
-    p = (j <= g.K) ? target + (b * (g.K + 1) + j) * g.V
-                   : draft + (b * g.K + (j - g.K - 1)) * g.V;
+    const int pos = w < 2 * g.np ? g.p0 + (w >> 1) : g.K;
+    const bool is_draft = w < 2 * g.np && (w & 1);
+    p = is_draft ? draft + (b * g.K + pos) * g.V : target + (b * (g.K + 1) + pos) * g.V;
     head = row_head(p, g.V);
     nvec = (g.V - head) / VEC;
     pv = reinterpret_cast<const uint4 *>(p + head);
   }
   __device__ __forceinline__ void start(const T *target, const T *draft, const StatsGeom &g,
                                         long long t) {
-    const int R = 2 * g.K + 1;
     row = t / g.tpr;
     ti = (int)(t - row * g.tpr);
-    b = row / R;
-    j = (int)(row - b * R);
+    b = row / g.rps;
+    w = (int)(row - b * g.rps);
     point(target, draft, g);
   }
   __device__ __forceinline__ void next_row(const T *target, const T *draft, const StatsGeom &g) {
     ++row;
     ti = 0;
-    if (++j == 2 * g.K + 1) {
-      j = 0;
+    if (++w == g.rps) {
+      w = 0;
       ++b;
     }
     point(target, draft, g);
@@ -450,6 +465,7 @@ __global__ void __launch_bounds__(NTS, kStatsCtasPerSm) k_row_stats(const T *__r
     rc.start(target, draft, g, t0);
     for (long long row = row_first; row <= row_last; ++row) {
       if (row != row_first) rc.next_row(target, draft, g);
+      if (!seq_active(g, rc.b)) continue;
       const int tb = (row == row_first) ? (int)(t0 - row * g.tpr) : 0;
       const int te = (row == row_last) ? (int)(t1 - row * g.tpr) : g.tpr;
       for (int ti = tb; ti < te; ++ti) {
@@ -495,7 +511,7 @@ __global__ void __launch_bounds__(NTS, kStatsCtasPerSm) k_row_stats(const T *__r
   float T_next = (rc.b + 1 < B) ? __ldg(temperature + rc.b + 1) : 1.0f;
   for (long long row = row_first; row <= row_last; ++row) {
     if (row != row_first) {
-      const bool new_seq = (rc.j == 2 * g.K);
+      const bool new_seq = (rc.w == g.rps - 1);
       rc.next_row(target, draft, g);
       if (new_seq) {
         c = make_scale(kLog2e / (double)T_next);
@@ -503,6 +519,7 @@ __global__ void __launch_bounds__(NTS, kStatsCtasPerSm) k_row_stats(const T *__r
         T_next = (rc.b + 1 < B) ? __ldg(temperature + rc.b + 1) : 1.0f;
       }
     }
+    if (!seq_active(g, rc.b)) continue;
     const int tb = (row == row_first) ? (int)(t0 - row * g.tpr) : 0;
     const int te = (row == row_last) ? (int)(t1 - row * g.tpr) : g.tpr;
     const long long full_tiles = rc.nvec / TV;  // tiles with all TV vectors
@@ -693,13 +710,29 @@ __device__ __noinline__ int draw_exact64(const T *pt, const T *pd, long long V, 
   return y;
 }
 
+// The window and decision state of a finish pass (the rows of StatsGeom's
+// window).  With `state` null the pass decides every sequence over its window
+// and draws.  Otherwise (early exit):
+//   decide-only pass: a sequence rejected inside the window gets its outputs
+//     (but the drawn token), state[b] = n and info[b]; one accepting the whole
+//     window gets the window's tokens and stays kSeqActive; an invalid one gets
+//     -1 outputs and state[b] = -1;
+//   final pass: a sequence decided earlier goes straight to its draw (from
+//     info[b]); an active one is tested on this window, then drawn.
+struct FinishWindow {
+  int p0, np, bonus, rps;
+  int decide_only;
+  int *state;
+  SeqInfo *info;
+};
+
 template <typename T, int UW>
 __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
     const T *__restrict__ target, const T *__restrict__ draft,
     const int32_t *__restrict__ tokens, const float *__restrict__ u_accept,
     const float *__restrict__ u_resample, const float *__restrict__ temperature, int K,
     long long V, int tpr, long long tiles, long long G1, int slots, int nsr, int cpb,
-    const Partial *__restrict__ part,
+    FinishWindow fw, const Partial *__restrict__ part,
     ResPartial *__restrict__ rpart, unsigned *__restrict__ counters,
     int32_t *__restrict__ out_tokens, int32_t *__restrict__ out_n,
     float *__restrict__ dbg_row_max, double *__restrict__ dbg_row_sum,
@@ -717,6 +750,7 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
   const long long b = (long long)blockIdx.x / ncb;
   const int cb = (int)((long long)blockIdx.x - b * ncb);  // this CTA: chunks cb*cpb ...
   const int R = 2 * K + 1;
+  const int RW = fw.rps;  // rows of the window per sequence
 
   // ---- inputs of this call (independent of the statistics kernel) ----
   const float Tf = __ldg(temperature + b);
@@ -725,109 +759,148 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
   int x = 0;
   bool x_ok = true;
   float zt_x = 0.f, zd_x = 0.f, u = 0.f;
-  if (warp == 0 && lane < K) {
-    x = __ldg(tokens + b * K + lane);
+  const int pos = fw.p0 + lane;  // the position lane `lane` of warp 0 tests
+  if (warp == 0 && lane < fw.np) {
+    x = __ldg(tokens + b * K + pos);
     x_ok = (x >= 0) && ((long long)x < V);
-    u = __ldg(u_accept + b * K + lane);
+    u = __ldg(u_accept + b * K + pos);
     if (x_ok) {
-      zt_x = Dt<T>::load(target + (b * (K + 1) + lane) * V + x);
-      zd_x = Dt<T>::load(draft + (b * K + lane) * V + x);
+      zt_x = Dt<T>::load(target + (b * (K + 1) + pos) * V + x);
+      zd_x = Dt<T>::load(draft + (b * K + pos) * V + x);
     }
   }
   const float ures = __ldg(u_resample + b);
   cudaGridDependencySynchronize();  // the row statistics are complete from here on
 
-  // ---- combine the V-split partials of every row (fp64) ----
-  for (int r = warp; r < R; r += NWARP) {
-    const long long row = b * R + r;
-    const Partial *P = part + row * slots * CW;
-    // partials of the CTAs of the statistics sweep that hold tiles of this
-    // row, in order, CW consumer warps each
-    const int nslot = (int)(tile_owner(row * tpr + tpr - 1, G1, tiles) -
-                            tile_owner(row * tpr, G1, tiles) + 1) * CW;
-    // first 32 partials in registers (one load per lane), the rest streamed
-    Partial p0;
-    p0.m = -INFINITY;
-    p0.s = 0.0;
-    if (lane < nslot) p0 = P[lane];
-    float m = p0.m;
-    for (int s = lane + 32; s < nslot; s += 32) m = fmaxf(m, P[s].m);
-    m = warp_max_nan(m);
-    double acc = (lane < nslot)
-                     ? ((p0.m == -INFINITY) ? p0.s : p0.s * exp2(((double)p0.m - (double)m) * c64))
-                     : 0.0;
-    for (int s = lane + 32; s < nslot; s += 32) {
-      const Partial ps = P[s];
-      acc += (ps.m == -INFINITY) ? ps.s : ps.s * exp2(((double)ps.m - (double)m) * c64);
-    }
-    acc = warp_sum(acc);
-    if (lane == 0) {
-      sM[r] = m;
-      sS[r] = acc;
-      if (cb == 0 && dbg_row_max) dbg_row_max[b * R + r] = m;
-      if (cb == 0 && dbg_row_sum) dbg_row_sum[b * R + r] = acc;
-    }
-  }
-  __syncthreads();
-
-  // ---- acceptance test and first rejection (warp 0) ----
-  if (warp == 0) {
-    // a timed-out wait in this call (or an earlier, unacknowledged one) makes
-    // every sequence invalid rather than silently wrong
-    const bool timed_out = (*(volatile unsigned *)&g_error_flags & SPECDEC_ERR_TIMEOUT) != 0;
-    bool rows_ok = true;
-    for (int r = lane; r < R; r += 32)
-      rows_ok = rows_ok && isfinite(sM[r]) && isfinite(sS[r]) && sS[r] > 0.0;
-    rows_ok = __all_sync(FULL, rows_ok) && !timed_out;
-    bool acc_i = false;
-    double p = 0.0, q = 0.0;
-    if (lane < K && x_ok && rows_ok && t_ok) {
-      p = exp2(((double)zt_x - (double)sM[lane]) * c64) / sS[lane];
-      q = exp2(((double)zd_x - (double)sM[K + 1 + lane]) * c64) / sS[K + 1 + lane];
-      acc_i = (double)u * q < p;
-    }
-    const unsigned bad_x = __ballot_sync(FULL, lane < K && !x_ok);
-    const unsigned accm = __ballot_sync(FULL, lane < K && acc_i);
-    const bool seq_ok = t_ok && rows_ok && bad_x == 0;
-    const unsigned kmask = (K >= 32) ? FULL : ((1u << K) - 1u);
-    const unsigned rej = ~accm & kmask;
-    const int n = seq_ok ? (rej ? __ffs(rej) - 1 : K) : -1;
-    if (lane == 0) s_n = n;
-    if (cb == 0) {
-      int32_t *ot = out_tokens + b * (K + 1);
-      if (!seq_ok) {
-        for (int i = lane; i <= K; i += 32) ot[i] = -1;
-      } else {
-        if (lane < n) ot[lane] = x;
-        for (int i = n + 1 + lane; i <= K; i += 32) ot[i] = -1;
-        if (lane < K && lane <= n) {
-          if (dbg_px) dbg_px[b * K + lane] = p;
-          if (dbg_qx) dbg_qx[b * K + lane] = q;
-        }
+  // (the decide-only pass is the first: every sequence is open there)
+  const int st_b = (fw.state && !fw.decide_only) ? __ldcg(fw.state + b) : kSeqActive;
+  if (st_b == -1) return;  // found invalid by an earlier pass: its outputs are written
+  int n;
+  float Mt, Md;
+  double St, Sd;
+  if (st_b >= 0) {
+    // decided by an earlier pass: straight to the draw
+    const SeqInfo *si = fw.info + b;
+    n = st_b;
+    Mt = __ldcg(&si->Mt);
+    Md = __ldcg(&si->Md);
+    St = __ldcg(&si->St);
+    Sd = __ldcg(&si->Sd);
+  } else {
+    // ---- combine the V-split partials of every row of the window (fp64) ----
+    for (int r = warp; r < RW; r += NWARP) {
+      const long long row = b * RW + r;
+      const Partial *P = part + row * slots * CW;
+      // partials of the CTAs of the statistics sweep that hold tiles of this
+      // row, in order, CW consumer warps each
+      const int nslot = (int)(tile_owner(row * tpr + tpr - 1, G1, tiles) -
+                              tile_owner(row * tpr, G1, tiles) + 1) * CW;
+      // first 32 partials in registers (one load per lane), the rest streamed
+      Partial p0;
+      p0.m = -INFINITY;
+      p0.s = 0.0;
+      if (lane < nslot) p0 = P[lane];
+      float m = p0.m;
+      for (int s = lane + 32; s < nslot; s += 32) m = fmax_nan(m, P[s].m);
+      m = warp_max_nan(m);
+      double acc =
+          (lane < nslot)
+              ? ((p0.m == -INFINITY) ? p0.s : p0.s * exp2(((double)p0.m - (double)m) * c64))
+              : 0.0;
+      for (int s = lane + 32; s < nslot; s += 32) {
+        const Partial ps = P[s];
+        acc += (ps.m == -INFINITY) ? ps.s : ps.s * exp2(((double)ps.m - (double)m) * c64);
       }
+      acc = warp_sum(acc);
       if (lane == 0) {
-        out_n[b] = n;
-        if (!seq_ok) {
-          unsigned f = 0;
-          if (!t_ok) f |= SPECDEC_ERR_TEMPERATURE;
-          if (bad_x) f |= SPECDEC_ERR_TOKEN;
-          if (!rows_ok) f |= SPECDEC_ERR_LOGITS;
-          atomicOr(&g_error_flags, f);
+        sM[r] = m;
+        sS[r] = acc;
+        // natural row index: target rows 0..K, then draft rows 0..K-1
+        const int rp = r < 2 * fw.np ? fw.p0 + (r >> 1) : K;
+        const int j = (r < 2 * fw.np && (r & 1)) ? K + 1 + rp : rp;
+        if (cb == 0 && dbg_row_max) dbg_row_max[b * R + j] = m;
+        if (cb == 0 && dbg_row_sum) dbg_row_sum[b * R + j] = acc;
+      }
+    }
+    __syncthreads();
+
+    // ---- acceptance test and first rejection (warp 0) ----
+    if (warp == 0) {
+      // a timed-out wait in this call (or an earlier, unacknowledged one) makes
+      // every sequence invalid rather than silently wrong
+      const bool timed_out = (*(volatile unsigned *)&g_error_flags & SPECDEC_ERR_TIMEOUT) != 0;
+      bool rows_ok = true;
+      for (int r = lane; r < RW; r += 32)
+        rows_ok = rows_ok && isfinite(sM[r]) && isfinite(sS[r]) && sS[r] > 0.0;
+      rows_ok = __all_sync(FULL, rows_ok) && !timed_out;
+      bool acc_i = false;
+      double p = 0.0, q = 0.0;
+      if (lane < fw.np && x_ok && rows_ok && t_ok) {
+        p = exp2(((double)zt_x - (double)sM[2 * lane]) * c64) / sS[2 * lane];
+        q = exp2(((double)zd_x - (double)sM[2 * lane + 1]) * c64) / sS[2 * lane + 1];
+        acc_i = (double)u * q < p;
+      }
+      const unsigned bad_x = __ballot_sync(FULL, lane < fw.np && !x_ok);
+      const unsigned accm = __ballot_sync(FULL, lane < fw.np && acc_i);
+      const bool seq_ok = t_ok && rows_ok && bad_x == 0;
+      const unsigned kmask = (fw.np >= 32) ? FULL : ((1u << fw.np) - 1u);
+      const unsigned rej = ~accm & kmask;
+      // the decision: rejected at n, all of K accepted (bonus), or still open
+      int nn = rej ? fw.p0 + __ffs(rej) - 1 : (fw.bonus ? K : kSeqActive);
+      if (!seq_ok) nn = -1;
+      if (lane == 0) s_n = nn;
+      if (cb == 0) {
+        int32_t *ot = out_tokens + b * (K + 1);
+        if (nn == -1) {
+          for (int i = lane; i <= K; i += 32) ot[i] = -1;
+        } else {
+          const int last = nn >= 0 ? nn : fw.p0 + fw.np;  // tokens accepted in the window
+          if (lane < fw.np && pos < last) ot[pos] = x;
+          if (nn >= 0)
+            for (int i = nn + 1 + lane; i <= K; i += 32) ot[i] = -1;
+          if (lane < fw.np && pos <= (nn >= 0 ? nn : K)) {
+            if (dbg_px) dbg_px[b * K + pos] = p;
+            if (dbg_qx) dbg_qx[b * K + pos] = q;
+          }
+        }
+        if (lane == 0) {
+          if (nn != kSeqActive) out_n[b] = nn;
+          if (fw.state) fw.state[b] = nn;
+          if (nn == -1) {
+            unsigned f = 0;
+            if (!t_ok) f |= SPECDEC_ERR_TEMPERATURE;
+            if (bad_x) f |= SPECDEC_ERR_TOKEN;
+            if (!rows_ok) f |= SPECDEC_ERR_LOGITS;
+            atomicOr(&g_error_flags, f);
+          }
+          if (fw.decide_only && nn >= 0) {  // the drawn pair for the final pass
+            const int wt = nn == K ? 2 * fw.np : 2 * (nn - fw.p0);
+            SeqInfo si;
+            si.Mt = sM[wt];
+            si.St = sS[wt];
+            si.Md = nn == K ? 0.f : sM[wt + 1];
+            si.Sd = nn == K ? 1.0 : sS[wt + 1];
+            fw.info[b] = si;
+          }
         }
       }
     }
+    __syncthreads();
+    n = s_n;
+    if (n < 0 || fw.decide_only) return;  // invalid, still open, or not drawn in this pass
+    const int wt = n == K ? 2 * fw.np : 2 * (n - fw.p0);
+    Mt = sM[wt];
+    St = sS[wt];
+    Md = n == K ? 0.f : sM[wt + 1];
+    Sd = n == K ? 1.0 : sS[wt + 1];
   }
-  __syncthreads();
-  const int n = s_n;
-  if (n < 0) return;  // invalid sequence (the same for every CTA of it)
 
   // ---- this CTA's chunk of the drawn row pair ----
   DrawRow d;
   d.bonus = (n == K);
-  d.Mt = sM[n];
-  const double St = sS[n];
-  d.Md = d.bonus ? 0.f : sM[K + 1 + n];
-  const double Sd = d.bonus ? 1.0 : sS[K + 1 + n];
+  d.Mt = Mt;
+  d.Md = d.bonus ? 0.f : Md;
+  if (d.bonus) Sd = 1.0;
   d.c = make_scale(c64);
   const double lam = d.bonus ? 0.0 : St / Sd;
   d.lhi = (float)lam;
@@ -1038,10 +1111,20 @@ std::unordered_map<int, DeviceBuf> g_staging;  // end-to-end staging per device
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-struct Plan {
-  int esize, vec, U, tpr, slots, nsr, cpb;
+// One statistics sweep: the window of positions it reads and its static
+// partition of tiles over CTAs.
+struct Sweep {
+  int p0, np, bonus, rps;
   long long rows, tiles, G1;  // G1: CTAs of the statistics sweep
-  size_t off_part, off_rpart, off_cnt, total;
+  int slots;                  // partial slots per row
+};
+
+struct Plan {
+  int esize, vec, U, tpr, nsr, cpb;
+  Sweep full;            // the whole batch, every row
+  Sweep first, second;   // early exit: positions [0, P), then [P, K] with the bonus row
+  int slots_max;
+  size_t off_part, off_rpart, off_cnt, off_state, off_info, total;
 };
 
 int num_sms() {
@@ -1050,6 +1133,25 @@ int num_sms() {
   return n > 0 ? n : 148;
 }
 
+Sweep make_sweep(int B, int p0, int np, int bonus, int tpr, long long cap) {
+  Sweep w;
+  w.p0 = p0;
+  w.np = np;
+  w.bonus = bonus;
+  w.rps = 2 * np + bonus;
+  w.rows = (long long)B * w.rps;
+  w.tiles = w.rows * tpr;
+  w.G1 = w.tiles < cap ? w.tiles : cap;
+  if (w.G1 < 1) w.G1 = 1;
+  // partial slots per row: the most CTAs whose tile ranges meet one row
+  const long long minr = w.tiles / w.G1;  // shortest range
+  w.slots = minr > 0 ? (int)((tpr - 1 + minr - 1) / minr + 1) : 1;
+  return w;
+}
+
+// Positions the first early-exit sweep reads: two (a sequence whose first two
+// draft tokens are both accepted goes on to the second sweep).
+inline int early_split(int K) { return K < 2 ? K : 2; }
 
 // Work decomposition for these sizes; a pure function of the sizes and the SM
 // count, so repeated calls reduce in the same order (bit-reproducible).
@@ -1058,24 +1160,26 @@ bool make_plan(int B, int K, int V, specdec_dtype dtype, int sms, Plan &pl) {
   if (dtype != SPECDEC_F32 && dtype != SPECDEC_BF16) return false;
   pl.esize = dtype == SPECDEC_BF16 ? 2 : 4;
   pl.vec = 16 / pl.esize;
-  pl.rows = (long long)B * (2 * K + 1);
+  const long long rows = (long long)B * (2 * K + 1);
   const long long nvec_max = ((long long)V + pl.vec - 1) / pl.vec;
   // tiles of 4 vectors per consumer thread (16 KB); 1 vector per thread when
   // 16 KB tiles would leave SMs idle (single-sequence batches)
   const long long cap = (long long)kStatsCtasPerSm * sms;
   long long tpr = (nvec_max + NTC * 4 - 1) / (NTC * 4);
   pl.U = 4;
-  if (pl.rows * tpr < 2 * cap) {
+  if (rows * tpr < 2 * cap) {
     pl.U = 1;
     tpr = (nvec_max + NTC - 1) / NTC;
   }
   if (tpr < 1) tpr = 1;
   pl.tpr = (int)tpr;
-  pl.tiles = pl.rows * tpr;
-  pl.G1 = pl.tiles < cap ? pl.tiles : cap;
-  // partial slots per row: the most CTAs whose tile ranges meet one row
-  const long long minr = pl.tiles / pl.G1;  // shortest range
-  pl.slots = (int)((tpr - 1 + minr - 1) / minr + 1);
+  pl.full = make_sweep(B, 0, K, 1, pl.tpr, cap);
+  const int P = early_split(K);
+  pl.first = make_sweep(B, 0, P, 0, pl.tpr, cap);
+  pl.second = make_sweep(B, P, K - P, 1, pl.tpr, cap);
+  pl.slots_max = pl.full.slots;
+  if (pl.first.slots > pl.slots_max) pl.slots_max = pl.first.slots;
+  if (pl.second.slots > pl.slots_max) pl.slots_max = pl.second.slots;
   // k_finish chunks: 32 lanes x kFinishUW vectors of the drawn row pair
   const long long nr = (nvec_max + 32LL * kFinishUW - 1) / (32LL * kFinishUW);
   pl.nsr = (int)(nr > 0 ? nr : 1);
@@ -1089,11 +1193,15 @@ bool make_plan(int B, int K, int V, specdec_dtype dtype, int sms, Plan &pl) {
   if ((long long)B * (K + 1) * (long long)V > (1LL << 56)) return false;
   size_t off = 0;
   pl.off_part = off;
-  off = align256(off + sizeof(Partial) * (size_t)pl.rows * pl.slots * CW);
+  off = align256(off + sizeof(Partial) * (size_t)rows * pl.slots_max * CW);
   pl.off_rpart = off;
   off = align256(off + sizeof(ResPartial) * (size_t)B * pl.nsr);
   pl.off_cnt = off;
   off = align256(off + sizeof(unsigned) * (size_t)B);
+  pl.off_state = off;
+  off = align256(off + sizeof(int) * (size_t)B);
+  pl.off_info = off;
+  off = align256(off + sizeof(SeqInfo) * (size_t)B);
   pl.total = off > 0 ? off : 256;
   return true;
 }
@@ -1161,11 +1269,15 @@ struct LaunchTimer {
   }
 };
 
+// One pass: a statistics sweep over `sw` (of the open sequences when `state`
+// is set and the pass is not the first), then k_finish over the same window
+// (programmatic dependent launch: its launch and gathers overlap the sweep).
 template <typename T>
-specdec_status launch_all(const void *tg, const void *dr, const int32_t *tok, const float *ua,
-                          const float *ur, const float *temp, int B, int K, int V,
-                          const Plan &pl, char *ws, const specdec_debug *dbg, int32_t *out_tokens,
-                          int32_t *out_n, cudaStream_t st) {
+specdec_status launch_pass(const void *tg, const void *dr, const int32_t *tok, const float *ua,
+                           const float *ur, const float *temp, int B, int K, int V,
+                           const Plan &pl, const Sweep &sw, int *state, SeqInfo *info,
+                           bool decide_only, char *ws, const specdec_debug *dbg,
+                           int32_t *out_tokens, int32_t *out_n, cudaStream_t st) {
   const T *t = static_cast<const T *>(tg);
   const T *d = static_cast<const T *>(dr);
   Partial *part = reinterpret_cast<Partial *>(ws + pl.off_part);
@@ -1175,8 +1287,12 @@ specdec_status launch_all(const void *tg, const void *dr, const int32_t *tok, co
   g.K = K;
   g.V = V;
   g.tpr = pl.tpr;
-  g.tiles = pl.tiles;
-  g.slots = pl.slots;
+  g.tiles = sw.tiles;
+  g.slots = sw.slots;
+  g.p0 = sw.p0;
+  g.np = sw.np;
+  g.rps = sw.rps;
+  g.state = decide_only ? nullptr : state;  // the first pass reads every sequence
   cudaError_t e = cudaSuccess;
   {
     LaunchTimer lt(KID_STATS, st);
@@ -1185,21 +1301,47 @@ specdec_status launch_all(const void *tg, const void *dr, const int32_t *tok, co
     // the sweep assumes its CTAs are co-resident only for speed, not for
     // progress: nothing waits on another CTA
     resident_ctas(kern, NTS, smem);
-    kern<<<(unsigned)pl.G1, NTS, smem, st>>>(t, d, temp, g, part, cnt, B);
+    kern<<<(unsigned)sw.G1, NTS, smem, st>>>(t, d, temp, g, part, cnt, B);
     e = cudaGetLastError();
   }
   if (e != cudaSuccess) return SPECDEC_ECUDA;
   {
     LaunchTimer lt(KID_FINISH, st);
-    const unsigned g2 = (unsigned)((long long)B * ((pl.nsr + pl.cpb - 1) / pl.cpb));
+    // a decide-only pass draws nothing: one CTA per sequence
+    const int cpb = decide_only ? pl.nsr : pl.cpb;
+    const unsigned g2 = (unsigned)((long long)B * ((pl.nsr + cpb - 1) / cpb));
+    FinishWindow fw;
+    fw.p0 = sw.p0;
+    fw.np = sw.np;
+    fw.bonus = sw.bonus;
+    fw.rps = sw.rps;
+    fw.decide_only = decide_only ? 1 : 0;
+    fw.state = state;
+    fw.info = info;
     auto kern = k_finish<T, kFinishUW>;
-    e = launch_pdl(kern, g2, NT, st, t, d, tok, ua, ur, temp, K, (long long)V, pl.tpr, pl.tiles,
-                   pl.G1, pl.slots, pl.nsr, pl.cpb,
-                   (const Partial *)part, rp, cnt, out_tokens, out_n,
-                   dbg ? dbg->row_max : nullptr, dbg ? dbg->row_sum : nullptr,
+    e = launch_pdl(kern, g2, NT, st, t, d, tok, ua, ur, temp, K, (long long)V, pl.tpr, sw.tiles,
+                   sw.G1, sw.slots, pl.nsr, cpb, fw, (const Partial *)part, rp, cnt, out_tokens,
+                   out_n, dbg ? dbg->row_max : nullptr, dbg ? dbg->row_sum : nullptr,
                    dbg ? dbg->p_x : nullptr, dbg ? dbg->q_x : nullptr, dbg ? dbg->Z : nullptr);
   }
   return e == cudaSuccess ? SPECDEC_OK : SPECDEC_ECUDA;
+}
+
+template <typename T>
+specdec_status launch_all(const void *tg, const void *dr, const int32_t *tok, const float *ua,
+                          const float *ur, const float *temp, int B, int K, int V,
+                          const Plan &pl, bool early_exit, char *ws, const specdec_debug *dbg,
+                          int32_t *out_tokens, int32_t *out_n, cudaStream_t st) {
+  if (!early_exit)
+    return launch_pass<T>(tg, dr, tok, ua, ur, temp, B, K, V, pl, pl.full, nullptr, nullptr,
+                          false, ws, dbg, out_tokens, out_n, st);
+  int *state = reinterpret_cast<int *>(ws + pl.off_state);
+  SeqInfo *info = reinterpret_cast<SeqInfo *>(ws + pl.off_info);
+  specdec_status s = launch_pass<T>(tg, dr, tok, ua, ur, temp, B, K, V, pl, pl.first, state,
+                                    info, true, ws, dbg, out_tokens, out_n, st);
+  if (s != SPECDEC_OK) return s;
+  return launch_pass<T>(tg, dr, tok, ua, ur, temp, B, K, V, pl, pl.second, state, info, false,
+                        ws, dbg, out_tokens, out_n, st);
 }
 
 specdec_status check_args(const void *tg, const void *dr, const int32_t *tok, const float *ua,
@@ -1222,17 +1364,17 @@ specdec_status check_args(const void *tg, const void *dr, const int32_t *tok, co
 specdec_status run(const void *tg, const void *dr, const int32_t *tok, const float *ua,
                    const float *ur, const float *temp, int B, int K, int V, specdec_dtype dtype,
                    void *ws, size_t ws_bytes, const specdec_debug *dbg, int32_t *ot, int32_t *on,
-                   cudaStream_t st) {
+                   cudaStream_t st, bool early_exit = false) {
   specdec_status s = check_args(tg, dr, tok, ua, ur, temp, B, K, V, dtype, ot, on);
   if (s != SPECDEC_OK || B == 0) return s;
   Plan pl;
   if (!make_plan(B, K, V, dtype, num_sms(), pl)) return SPECDEC_EINVAL;
   if (!ws || ws_bytes < pl.total || (reinterpret_cast<uintptr_t>(ws) & 255)) return SPECDEC_EINVAL;
   if (dtype == SPECDEC_BF16)
-    return launch_all<__nv_bfloat16>(tg, dr, tok, ua, ur, temp, B, K, V, pl,
+    return launch_all<__nv_bfloat16>(tg, dr, tok, ua, ur, temp, B, K, V, pl, early_exit,
                                      static_cast<char *>(ws), dbg, ot, on, st);
-  return launch_all<float>(tg, dr, tok, ua, ur, temp, B, K, V, pl, static_cast<char *>(ws), dbg,
-                           ot, on, st);
+  return launch_all<float>(tg, dr, tok, ua, ur, temp, B, K, V, pl, early_exit,
+                           static_cast<char *>(ws), dbg, ot, on, st);
 }
 
 // grow-only device buffer of the current device (zero-filled when (re)allocated)
@@ -1339,6 +1481,37 @@ specdec_status specdec_verify(const void *target_logits, const void *draft_logit
   return run(target_logits, draft_logits, draft_tokens, u_accept, u_resample, temperature, B, K,
              V, dtype, ws, need, nullptr, out_tokens, out_num_accepted,
              static_cast<cudaStream_t>(stream));
+}
+
+specdec_status specdec_verify_early_exit_ex(const void *target_logits, const void *draft_logits,
+                                            const int32_t *draft_tokens, const float *u_accept,
+                                            const float *u_resample, const float *temperature,
+                                            int B, int K, int V, specdec_dtype dtype,
+                                            void *workspace, size_t workspace_bytes,
+                                            const specdec_debug *dbg, int32_t *out_tokens,
+                                            int32_t *out_num_accepted, void *stream) {
+  return run(target_logits, draft_logits, draft_tokens, u_accept, u_resample, temperature, B, K,
+             V, dtype, workspace, workspace_bytes, dbg, out_tokens, out_num_accepted,
+             static_cast<cudaStream_t>(stream), true);
+}
+
+specdec_status specdec_verify_early_exit(const void *target_logits, const void *draft_logits,
+                                         const int32_t *draft_tokens, const float *u_accept,
+                                         const float *u_resample, const float *temperature,
+                                         int B, int K, int V, specdec_dtype dtype,
+                                         int32_t *out_tokens, int32_t *out_num_accepted,
+                                         void *stream) {
+  specdec_status s = check_args(target_logits, draft_logits, draft_tokens, u_accept, u_resample,
+                                temperature, B, K, V, dtype, out_tokens, out_num_accepted);
+  if (s != SPECDEC_OK || B == 0) return s;
+  const size_t need = specdec_workspace_bytes(B, K, V, dtype);
+  if (need == 0) return SPECDEC_EINVAL;
+  void *ws = nullptr;
+  s = ensure_buf(g_ws, need, static_cast<cudaStream_t>(stream), &ws);
+  if (s != SPECDEC_OK) return s;
+  return run(target_logits, draft_logits, draft_tokens, u_accept, u_resample, temperature, B, K,
+             V, dtype, ws, need, nullptr, out_tokens, out_num_accepted,
+             static_cast<cudaStream_t>(stream), true);
 }
 
 specdec_status specdec_verify_bf16(const void *target_logits, const void *draft_logits,

@@ -42,8 +42,9 @@ def to_device(x):
         temperature=torch.from_numpy(x.temperature).to(dev))
 
 
-def gpu_verify(x, debug=True, dev_inputs=None, garbage_workspace=False):
-    """CUDA path through specdec_verify_ex (with diagnostics) or specdec_verify."""
+def gpu_verify(x, debug=True, dev_inputs=None, garbage_workspace=False, early_exit=False):
+    """CUDA path through specdec_verify_ex (with diagnostics) or specdec_verify
+    (their early-exit forms with ``early_exit``)."""
     torch = require_cuda()
     d = dev_inputs if dev_inputs is not None else to_device(x)
     B, K = x.B, x.K
@@ -62,13 +63,13 @@ def gpu_verify(x, debug=True, dev_inputs=None, garbage_workspace=False):
             n = sd.specdec_workspace_bytes(B, K, x.V, dt)
             ws = torch.randint(0, 255, (n,), dtype=torch.uint8, device=dev)
         ot, on = sd.verify(d["target"], d["draft"], d["tokens"], d["u_accept"], d["u_resample"],
-                           d["temperature"], debug=dbg, workspace=ws)
+                           d["temperature"], debug=dbg, workspace=ws, early_exit=early_exit)
         torch.cuda.synchronize()
         for k, v in dbg.items():
             out[k] = v.cpu().numpy()
     else:
         ot, on = sd.verify(d["target"], d["draft"], d["tokens"], d["u_accept"], d["u_resample"],
-                           d["temperature"])
+                           d["temperature"], early_exit=early_exit)
         torch.cuda.synchronize()
     out["out_tokens"] = ot.cpu().numpy()
     out["num_accepted"] = on.cpu().numpy()
@@ -91,12 +92,28 @@ def rel(a, b):
     return np.abs(a - b) / np.maximum(np.abs(b), 1e-200)
 
 
-def compare(g: dict, o: dict, seqs=None, rtol=RTOL, band=BAND, stats=True) -> dict:
+def rows_read(o: dict, early_split) -> np.ndarray:
+    """[B, 2K+1] mask of the rows a call reads: all of them, or with early exit
+    (first sweep over positions < early_split) those of positions < early_split
+    plus every row of the sequences that accepted all of those."""
+    on = o["num_accepted"]
+    B, K1 = o["out_tokens"].shape
+    K = K1 - 1
+    j = np.arange(2 * K + 1)
+    pos = np.where(j <= K, j, j - K - 1)
+    if early_split is None:
+        return np.ones((B, 2 * K + 1), bool)
+    return (pos[None, :] < early_split) | (on[:, None] >= early_split)
+
+
+def compare(g: dict, o: dict, seqs=None, rtol=RTOL, band=BAND, stats=True,
+            early_split=None) -> dict:
     """Element-by-element comparison of the CUDA path (g) with the oracle (o).
 
     Integer outputs: bit-exact on every sequence whose oracle decisions are not
     within ``band`` of a threshold; such boundary draws are counted.  Invalid
-    sequences (n = -1) must agree exactly.  Probabilities: within ``rtol``."""
+    sequences (n = -1) must agree exactly.  Probabilities: within ``rtol``, on
+    the rows the call reads (``early_split``: see rows_read)."""
     if seqs is not None:
         g = {k: v[np.asarray(seqs)] for k, v in g.items()}
     on, gn = o["num_accepted"], g["num_accepted"]
@@ -120,11 +137,11 @@ def compare(g: dict, o: dict, seqs=None, rtol=RTOL, band=BAND, stats=True) -> di
     assert res["mismatched"] <= int(1e-4 * draws), res
     if not stats or "row_sum" not in g:
         return res
-    v = valid
+    v = valid[:, None] & rows_read(o, early_split)
     assert np.array_equal(g["row_max"][v].astype(np.float64), o["row_max"][v]), "row max"
     e_s = rel(g["row_sum"][v], o["row_sum"][v])
     assert e_s.max(initial=0) <= rtol, ("row sum", e_s.max())
-    same = exact | (v & (gn == on))
+    same = exact | (valid & (gn == on))
     reach = (np.arange(K)[None, :] <= on[:, None]) & same[:, None]
     e_p = rel(g["p_x"][reach], o["p_x"][reach])
     e_q = rel(g["q_x"][reach], o["q_x"][reach])
