@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--kernel-timing", choices=["on", "off"], default="on")
     ap.add_argument("--early-exit", choices=["on", "off"], default="on",
                     help="also time specdec_verify_early_exit on the same steps")
+    ap.add_argument("--smc", choices=["on", "off"], default="on",
+                    help="also time specdec_smc_step (groups of 8 particles) on the same steps")
     return ap.parse_args()
 
 
@@ -352,6 +354,43 @@ def run_cuda(args):
                  "note": "value counts the full two-tensor floor per step, as the headline "
                          "does; read_GBs counts the rows this call actually reads"}
 
+    # ---- SMC-SD weight step on the same logits (groups of 8 particles) -------
+    smc_line = None
+    if args.smc == "on" and B % 8 == 0:
+        Np = 8
+        G = B // Np
+        ur_g = torch.full((G,), 0.5, dtype=torch.float32, device=dev)
+        lw_out = torch.empty((B,), dtype=torch.float64, device=dev)
+        ess_o = torch.empty((G,), dtype=torch.float64, device=dev)
+        anc = torch.empty((B,), dtype=torch.int32, device=dev)
+        fs = L.specdec_smc_step
+
+        def smc(i):
+            b = bufs[i % ncopies]
+            return fs(b["t"].data_ptr(), b["d"].data_ptr(), b["tok"].data_ptr(),
+                      b["ur"].data_ptr(), b["T"].data_ptr(), None, ur_g.data_ptr(), 0.5, B, Np,
+                      K, V, dt_code, b["ot"].data_ptr(), lw_out.data_ptr(), ess_o.data_ptr(),
+                      anc.data_ptr(), None, sp)
+        for i in range(3):
+            if smc(i) != 0:
+                raise RuntimeError("specdec_smc_step failed")
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for i in range(args.steps):
+            smc(i)
+        s1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms_smc = sdist.max_over_ranks(s0.elapsed_time(s1), dev) / args.steps
+        smc_line = {"ms_per_step": ms_smc, "value": total_bytes / (ms_smc * 1e-3) / 1e9,
+                    "unit": "GB/s", "particles_per_group": Np, "groups": G * world,
+                    "note": "one SMC-SD round over the same logits: statistics sweep, log "
+                            "importance ratios and bonus draws, ESS and systematic resampling"}
+
     # ---- end to end through the host entry point (pinned buffers) ----------
     pin = {k: torch.from_numpy(np.ascontiguousarray(getattr(x, k))).pin_memory()
            for k in ("target", "draft", "tokens", "u_accept", "u_resample", "temperature")}
@@ -416,6 +455,8 @@ def run_cuda(args):
         line["kernel_us"] = {k: (v[0] / max(v[1], 1) * 1e3) for k, v in kern.items()}
     if early is not None:
         line["early_exit"] = early
+    if smc_line is not None:
+        line["smc_step"] = smc_line
     line["e2e"] = {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                    "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
     line["clocks"] = sampler.summary()

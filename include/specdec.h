@@ -174,6 +174,42 @@ specdec_status specdec_verify_early_exit_ex(const void *target_logits, const voi
                                             const specdec_debug *dbg, int32_t *out_tokens,
                                             int32_t *out_num_accepted, void *stream);
 
+/* SMC-SD weight step (the SMC-SD page "Faster LLM Inference via Sequential
+ * Monte Carlo", section 2, "Methodology" and "Key differences from standard
+ * SD"): N draft particles per group extend their sequences by K draft tokens;
+ * the target scores all N x (K+1) positions; no token is rejected.  For each
+ * particle b (B = G*N particles, G groups of N consecutive particles):
+ *   out_tokens[b, 0..K-1] = draft_tokens[b, :] and out_tokens[b, K] = the
+ *     bonus token drawn from p_K = softmax(target_logits[b, K, :] / T_b) with
+ *     u_bonus[b] by the inverse-CDF rule of specdec_verify;
+ *   log_weight_increment[b] = sum_i [log p_i(x_i) - log q_i(x_i)] (fp64;
+ *     p_i, q_i the temperature softmaxes of target and draft row i);
+ *   log w = log_weights_in[b] (0 when log_weights_in is NULL) + increment.
+ * Per group g: normalised weights wbar = exp(log w - max) / sum, ess[g] =
+ * 1 / sum wbar^2 (fp64).  If ess[g] < ess_threshold * N the group is
+ * resampled systematically with the single uniform u_resample[g]:
+ * ancestors[g*N + k] = min{j : C_j > (k + u)/N} (C the running sum of wbar in
+ * particle order; an index within the group) and log_weights_out = 0;
+ * otherwise ancestors[g*N + k] = k and log_weights_out = log w.  The caller
+ * applies the ancestors to its particle state (e.g. KV-cache pages).
+ * Layouts: logits, tokens, temperature as in specdec_verify; u_bonus [B],
+ * log_weights_in / log_weights_out / log_weight_increment [B] fp64 (in and
+ * increment nullable; out may alias in), u_resample [G], ess [G] fp64,
+ * ancestors [B] int32.  Device memory, asynchronous on `stream`, library-owned
+ * workspace (as specdec_verify).
+ * Errors: SPECDEC_EINVAL for B not a multiple of N, N outside [1, 4096],
+ * ess_threshold negative or not finite, and the argument errors of
+ * specdec_verify.  A particle with an invalid input gets tokens -1 and log
+ * weight -inf (weight 0) and sets the device error word; a group whose
+ * particles are all invalid gets ess 0 and ancestors -1. */
+specdec_status specdec_smc_step(const void *target_logits, const void *draft_logits,
+                                const int32_t *draft_tokens, const float *u_bonus,
+                                const float *temperature, const double *log_weights_in,
+                                const float *u_resample, double ess_threshold, int B, int N,
+                                int K, int V, specdec_dtype dtype, int32_t *out_tokens,
+                                double *log_weights_out, double *ess, int32_t *ancestors,
+                                double *log_weight_increment, void *stream);
+
 /* End-to-end variant: every pointer is HOST memory (pinned memory makes the
  * copies asynchronous).  Copies the inputs to library-owned device buffers,
  * runs the verify step on `stream`, copies the outputs back and synchronises

@@ -36,6 +36,8 @@ _SIGS = {
     "specdec_verify_early_exit_ex": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P,
                                           ctypes.c_size_t, _P, _P, _P, _P]),
     "specdec_verify_static": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P]),
+    "specdec_smc_step": (_I, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_double, _I, _I, _I, _I, _I,
+                              _P, _P, _P, _P, _P, _P]),
     "specdec_device_errors": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
     "specdec_release": (None, []),
     "specdec_status_string": (ctypes.c_char_p, [_I]),
@@ -147,6 +149,47 @@ def specdec_verify_static(target, draft, tokens, u_accept, u_resample, temperatu
     for the size limit and the no-overlap rule)."""
     return lib().specdec_verify_static(target, draft, tokens, u_accept, u_resample, temperature,
                                        B, K, V, dtype, out_tokens, out_num_accepted, stream)
+
+
+def specdec_smc_step(target, draft, tokens, u_bonus, temperature, log_weights_in, u_resample,
+                     ess_threshold, B, N, K, V, dtype, out_tokens, log_weights_out, ess,
+                     ancestors, log_weight_increment, stream) -> int:
+    return lib().specdec_smc_step(target, draft, tokens, u_bonus, temperature, log_weights_in,
+                                  u_resample, float(ess_threshold), B, N, K, V, dtype,
+                                  out_tokens, log_weights_out, ess, ancestors,
+                                  log_weight_increment, stream)
+
+
+def smc_step(target, draft, tokens, u_bonus, temperature, u_resample, N, ess_threshold=0.5,
+             log_weights_in=None, stream=None) -> dict:
+    """One SMC-SD round on CUDA tensors (see specdec_smc_step): target
+    [B,K+1,V], draft [B,K,V], tokens [B,K] int32, u_bonus [B] / temperature [B]
+    float32, u_resample [B//N] float32, log_weights_in [B] float64 or None.
+    Returns a dict of CUDA tensors: out_tokens, log_weights, ess, ancestors,
+    increment."""
+    import torch
+    B, K1, V = target.shape
+    K = K1 - 1
+    if B % N:
+        raise ValueError("B must be a multiple of N")
+    dev = target.device
+    out = dict(out_tokens=torch.empty((B, K + 1), dtype=torch.int32, device=dev),
+               log_weights=torch.empty((B,), dtype=torch.float64, device=dev),
+               ess=torch.empty((B // N,), dtype=torch.float64, device=dev),
+               ancestors=torch.empty((B,), dtype=torch.int32, device=dev),
+               increment=torch.empty((B,), dtype=torch.float64, device=dev))
+    _check_dev(target, draft, tokens, u_bonus, temperature, u_resample)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    st = specdec_smc_step(target.data_ptr(), draft.data_ptr(), tokens.data_ptr(),
+                          u_bonus.data_ptr(), temperature.data_ptr(),
+                          None if log_weights_in is None else log_weights_in.data_ptr(),
+                          u_resample.data_ptr(), ess_threshold, B, N, K, V, _dtype_code(target),
+                          out["out_tokens"].data_ptr(), out["log_weights"].data_ptr(),
+                          out["ess"].data_ptr(), out["ancestors"].data_ptr(),
+                          out["increment"].data_ptr(), stream)
+    _chk(st, "specdec_smc_step")
+    return out
 
 
 def specdec_device_errors(stream=None) -> tuple:

@@ -719,11 +719,17 @@ __device__ __noinline__ int draw_exact64(const T *pt, const T *pd, long long V, 
 //     -1 outputs and state[b] = -1;
 //   final pass: a sequence decided earlier goes straight to its draw (from
 //     info[b]); an active one is tested on this window, then drawn.
+//
+// SMC-SD mode (`dlogw` set; the SMC-SD page, section 2): no token is rejected;
+// every particle keeps its K draft tokens, draws its bonus token from p_K, and
+// gets the log importance ratio of its K tokens,
+// dlogw[b] = sum_i [log p_i(x_i) - log q_i(x_i)] in fp64 (-inf when invalid).
 struct FinishWindow {
   int p0, np, bonus, rps;
   int decide_only;
   int *state;
   SeqInfo *info;
+  double *dlogw;
 };
 
 template <typename T, int UW>
@@ -763,7 +769,7 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
   if (warp == 0 && lane < fw.np) {
     x = __ldg(tokens + b * K + pos);
     x_ok = (x >= 0) && ((long long)x < V);
-    u = __ldg(u_accept + b * K + pos);
+    u = fw.dlogw ? 0.f : __ldg(u_accept + b * K + pos);  // (SMC-SD accepts no test)
     if (x_ok) {
       zt_x = Dt<T>::load(target + (b * (K + 1) + pos) * V + x);
       zd_x = Dt<T>::load(draft + (b * K + pos) * V + x);
@@ -844,7 +850,19 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
       const unsigned accm = __ballot_sync(FULL, lane < fw.np && acc_i);
       const bool seq_ok = t_ok && rows_ok && bad_x == 0;
       const unsigned kmask = (fw.np >= 32) ? FULL : ((1u << fw.np) - 1u);
-      const unsigned rej = ~accm & kmask;
+      unsigned rej = ~accm & kmask;
+      if (fw.dlogw) {
+        // SMC-SD: keep every draft token; weight by the log ratio of the window
+        double lr = 0.0;
+        if (lane < fw.np && seq_ok) {
+          const double iT = 1.0 / (double)Tf;
+          lr = (((double)zt_x - (double)sM[2 * lane]) * iT - log(sS[2 * lane])) -
+               (((double)zd_x - (double)sM[2 * lane + 1]) * iT - log(sS[2 * lane + 1]));
+        }
+        lr = warp_sum(lr);
+        if (cb == 0 && lane == 0) fw.dlogw[b] = seq_ok ? lr : -INFINITY;
+        rej = 0u;
+      }
       // the decision: rejected at n, all of K accepted (bonus), or still open
       int nn = rej ? fw.p0 + __ffs(rej) - 1 : (fw.bonus ? K : kSeqActive);
       if (!seq_ok) nn = -1;
@@ -1089,10 +1107,140 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
 }
 
 // ---------------------------------------------------------------------------
+// kernel 3 (SMC-SD): weights, effective sample size, systematic resampling
+// ---------------------------------------------------------------------------
+// One CTA per group of N particles (the SMC-SD page, section 2: "if the
+// effective sample size falls below a threshold, low-weight particles are
+// dropped and high-weight ones copied").  log w_n = log w_n(before) +
+// dlogw_n; normalised weights wbar = exp(log w - max) / sum, ESS =
+// 1 / sum wbar^2, all in fp64.  When ESS < threshold * N: systematic
+// resampling with the group's uniform u, ancestor a_k = min{j : C_j > (k+u)/N}
+// with C the inclusive running sum of wbar in particle order (a block scan,
+// contiguous particles per thread), found by binary search; every log-weight
+// of the group becomes 0.  Otherwise a_k = k and the log-weights carry over.
+// A group whose particles are all invalid (log-weight -inf) gets ESS 0,
+// ancestors -1 and log-weights -inf.
+constexpr int kSmcMaxN = 4096;  // particles per group (shared-memory running sums)
+
+__global__ void __launch_bounds__(NT) k_smc_resample(const double *__restrict__ dlogw,
+                                                     const double *__restrict__ logw_in,
+                                                     const float *__restrict__ u_resample,
+                                                     double ess_threshold, int N,
+                                                     double *__restrict__ logw_out,
+                                                     double *__restrict__ ess_out,
+                                                     int32_t *__restrict__ ancestors) {
+  extern __shared__ double sC[];  // N running sums
+  __shared__ double s_red[NWARP];
+  __shared__ int s_res;
+  const int g = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  cudaGridDependencySynchronize();  // the increments of this call are written
+  const long long base = (long long)g * N;
+  const int per = (N + NT - 1) / NT;  // contiguous particles per thread
+  const int k0 = tid * per < N ? tid * per : N;
+  const int k1 = k0 + per < N ? k0 + per : N;
+  auto lw = [&](int k) -> double {
+    const double a = __ldcg(dlogw + base + k);
+    return logw_in ? __ldcg(logw_in + base + k) + a : a;
+  };
+  // max
+  double m = -INFINITY;
+  for (int k = k0; k < k1; ++k) m = fmax(m, lw(k));
+#pragma unroll
+  for (int o = 16; o; o >>= 1) m = fmax(m, __shfl_xor_sync(FULL, m, o));
+  if (lane == 0) s_red[warp] = m;
+  __syncthreads();
+  m = s_red[0];
+  for (int w = 1; w < NWARP; ++w) m = fmax(m, s_red[w]);
+  __syncthreads();
+  if (!(m > -INFINITY) || !isfinite(m)) {  // every particle invalid (or NaN)
+    for (int k = tid; k < N; k += NT) {
+      logw_out[base + k] = -INFINITY;
+      ancestors[base + k] = -1;
+    }
+    if (tid == 0) ess_out[g] = 0.0;
+    return;
+  }
+  // weights relative to the max, their exclusive prefix (contiguous per thread)
+  double sw = 0.0;
+  for (int k = k0; k < k1; ++k) {
+    const double w = exp(lw(k) - m);
+    sC[k] = w;
+    sw += w;
+  }
+  double incl = sw;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double y = __shfl_up_sync(FULL, incl, o);
+    if (lane >= o) incl += y;
+  }
+  double excl = __shfl_up_sync(FULL, incl, 1);
+  if (lane == 0) excl = 0.0;
+  if (lane == 31) s_red[warp] = incl;
+  __syncthreads();
+  double before = 0.0, S = 0.0;
+  for (int w = 0; w < NWARP; ++w) {
+    if (w < warp) before += s_red[w];
+    S += s_red[w];
+  }
+  excl += before;
+  __syncthreads();
+  // normalised running sums and the sum of squares
+  double sq = 0.0, C = excl;
+  for (int k = k0; k < k1; ++k) {
+    const double wb = sC[k] / S;
+    sq += wb * wb;
+    C += sC[k];
+    sC[k] = C / S;
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) sq += __shfl_xor_sync(FULL, sq, o);
+  if (lane == 0) s_red[warp] = sq;
+  __syncthreads();
+  double q2 = 0.0;
+  for (int w = 0; w < NWARP; ++w) q2 += s_red[w];
+  const double ess = 1.0 / q2;
+  if (tid == 0) {
+    ess_out[g] = ess;
+    s_res = ess < ess_threshold * (double)N;
+  }
+  __syncthreads();
+  if (!s_res) {
+    for (int k = tid; k < N; k += NT) {
+      logw_out[base + k] = lw(k);
+      ancestors[base + k] = k;
+    }
+    return;
+  }
+  // last particle with positive weight (for targets rounding leaves past C)
+  int lastpos = -1;
+  for (int k = k0; k < k1; ++k)
+    if (sC[k] > (k > 0 ? sC[k - 1] : 0.0)) lastpos = k;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) lastpos = max(lastpos, __shfl_xor_sync(FULL, lastpos, o));
+  __shared__ int s_last[NWARP];
+  if (lane == 0) s_last[warp] = lastpos;
+  __syncthreads();
+  for (int w = 0; w < NWARP; ++w) lastpos = max(lastpos, s_last[w]);
+  const double u = (double)__ldg(u_resample + g);
+  for (int k = tid; k < N; k += NT) {
+    const double t = ((double)k + u) / (double)N;
+    int lo = 0, hi = N;  // first j with C_j > t, in [0, N]
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (sC[mid] > t) hi = mid;
+      else lo = mid + 1;
+    }
+    ancestors[base + k] = lo < N ? lo : lastpos;
+    logw_out[base + k] = 0.0;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-enum KernelId { KID_STATS = 0, KID_FINISH = 1, KID_COUNT = 2 };
-const char *kKernelNames[KID_COUNT] = {"k_row_stats", "k_finish"};
+enum KernelId { KID_STATS = 0, KID_FINISH = 1, KID_SMC = 2, KID_COUNT = 3 };
+const char *kKernelNames[KID_COUNT] = {"k_row_stats", "k_finish", "k_smc_resample"};
 
 std::mutex g_mu;
 uint64_t g_launches[KID_COUNT];
@@ -1124,7 +1272,7 @@ struct Plan {
   Sweep full;            // the whole batch, every row
   Sweep first, second;   // early exit: positions [0, P), then [P, K] with the bonus row
   int slots_max;
-  size_t off_part, off_rpart, off_cnt, off_state, off_info, total;
+  size_t off_part, off_rpart, off_cnt, off_state, off_info, off_dlogw, total;
 };
 
 int num_sms() {
@@ -1202,6 +1350,8 @@ bool make_plan(int B, int K, int V, specdec_dtype dtype, int sms, Plan &pl) {
   off = align256(off + sizeof(int) * (size_t)B);
   pl.off_info = off;
   off = align256(off + sizeof(SeqInfo) * (size_t)B);
+  pl.off_dlogw = off;
+  off = align256(off + sizeof(double) * (size_t)B);
   pl.total = off > 0 ? off : 256;
   return true;
 }
@@ -1277,7 +1427,8 @@ specdec_status launch_pass(const void *tg, const void *dr, const int32_t *tok, c
                            const float *ur, const float *temp, int B, int K, int V,
                            const Plan &pl, const Sweep &sw, int *state, SeqInfo *info,
                            bool decide_only, char *ws, const specdec_debug *dbg,
-                           int32_t *out_tokens, int32_t *out_n, cudaStream_t st) {
+                           int32_t *out_tokens, int32_t *out_n, cudaStream_t st,
+                           double *dlogw = nullptr) {
   const T *t = static_cast<const T *>(tg);
   const T *d = static_cast<const T *>(dr);
   Partial *part = reinterpret_cast<Partial *>(ws + pl.off_part);
@@ -1318,6 +1469,7 @@ specdec_status launch_pass(const void *tg, const void *dr, const int32_t *tok, c
     fw.decide_only = decide_only ? 1 : 0;
     fw.state = state;
     fw.info = info;
+    fw.dlogw = dlogw;
     auto kern = k_finish<T, kFinishUW>;
     e = launch_pdl(kern, g2, NT, st, t, d, tok, ua, ur, temp, K, (long long)V, pl.tpr, sw.tiles,
                    sw.G1, sw.slots, pl.nsr, cpb, fw, (const Partial *)part, rp, cnt, out_tokens,
@@ -1375,6 +1527,56 @@ specdec_status run(const void *tg, const void *dr, const int32_t *tok, const flo
                                      static_cast<char *>(ws), dbg, ot, on, st);
   return launch_all<float>(tg, dr, tok, ua, ur, temp, B, K, V, pl, early_exit,
                            static_cast<char *>(ws), dbg, ot, on, st);
+}
+
+// One SMC-SD round: the statistics sweep over every row, k_finish in SMC-SD
+// mode (log ratios, bonus draws), then k_smc_resample per group.
+specdec_status run_smc(const void *tg, const void *dr, const int32_t *tok, const float *ub,
+                       const float *temp, const double *lw_in, const float *ur, double thr,
+                       int B, int N, int K, int V, specdec_dtype dtype, void *ws,
+                       int32_t *ot, double *lw_out, double *ess, int32_t *anc, double *dlw,
+                       cudaStream_t st) {
+  if (B < 0 || N < 1 || N > kSmcMaxN || K < 1 || K > 32 || V < 1) return SPECDEC_EINVAL;
+  if (dtype != SPECDEC_F32 && dtype != SPECDEC_BF16) return SPECDEC_EINVAL;
+  if (B % N != 0 || !(thr >= 0.0) || !isfinite(thr)) return SPECDEC_EINVAL;
+  if (B == 0) return SPECDEC_OK;
+  if (!tg || !dr || !tok || !ub || !temp || !ur || !ot || !lw_out || !ess || !anc || !ws)
+    return SPECDEC_EINVAL;
+  const uintptr_t es = dtype == SPECDEC_BF16 ? 2 : 4;
+  if ((reinterpret_cast<uintptr_t>(tg) % es) || (reinterpret_cast<uintptr_t>(dr) % es))
+    return SPECDEC_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(tok) | reinterpret_cast<uintptr_t>(ub) |
+       reinterpret_cast<uintptr_t>(ur) | reinterpret_cast<uintptr_t>(temp) |
+       reinterpret_cast<uintptr_t>(ot) | reinterpret_cast<uintptr_t>(anc)) % 4)
+    return SPECDEC_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(lw_in) | reinterpret_cast<uintptr_t>(lw_out) |
+       reinterpret_cast<uintptr_t>(ess) | reinterpret_cast<uintptr_t>(dlw)) % 8)
+    return SPECDEC_EINVAL;
+  Plan pl;
+  if (!make_plan(B, K, V, dtype, num_sms(), pl)) return SPECDEC_EINVAL;
+  char *w = static_cast<char *>(ws);
+  int32_t *n_scratch = reinterpret_cast<int32_t *>(w + pl.off_state);
+  double *inc = dlw ? dlw : reinterpret_cast<double *>(w + pl.off_dlogw);
+  specdec_status s = (dtype == SPECDEC_BF16)
+      ? launch_pass<__nv_bfloat16>(tg, dr, tok, nullptr, ub, temp, B, K, V, pl, pl.full,
+                                   nullptr, nullptr, false, w, nullptr, ot, n_scratch, st, inc)
+      : launch_pass<float>(tg, dr, tok, nullptr, ub, temp, B, K, V, pl, pl.full, nullptr,
+                           nullptr, false, w, nullptr, ot, n_scratch, st, inc);
+  if (s != SPECDEC_OK) return s;
+  LaunchTimer lt(KID_SMC, st);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(B / N));
+  cfg.blockDim = dim3(NT);
+  cfg.dynamicSmemBytes = sizeof(double) * (size_t)N;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_smc_resample, (const double *)inc, lw_in, ur,
+                                           thr, N, lw_out, ess, anc);
+  return e == cudaSuccess ? SPECDEC_OK : SPECDEC_ECUDA;
 }
 
 // grow-only device buffer of the current device (zero-filled when (re)allocated)
@@ -1512,6 +1714,26 @@ specdec_status specdec_verify_early_exit(const void *target_logits, const void *
   return run(target_logits, draft_logits, draft_tokens, u_accept, u_resample, temperature, B, K,
              V, dtype, ws, need, nullptr, out_tokens, out_num_accepted,
              static_cast<cudaStream_t>(stream), true);
+}
+
+specdec_status specdec_smc_step(const void *target_logits, const void *draft_logits,
+                                const int32_t *draft_tokens, const float *u_bonus,
+                                const float *temperature, const double *log_weights_in,
+                                const float *u_resample, double ess_threshold, int B, int N,
+                                int K, int V, specdec_dtype dtype, int32_t *out_tokens,
+                                double *log_weights_out, double *ess, int32_t *ancestors,
+                                double *log_weight_increment, void *stream) {
+  if (B < 0 || N < 1 || K < 1 || K > 32 || V < 1) return SPECDEC_EINVAL;
+  if (B == 0) return SPECDEC_OK;
+  const size_t need = specdec_workspace_bytes(B, K, V, dtype);
+  if (need == 0) return SPECDEC_EINVAL;
+  void *ws = nullptr;
+  specdec_status s = ensure_buf(g_ws, need, static_cast<cudaStream_t>(stream), &ws);
+  if (s != SPECDEC_OK) return s;
+  return run_smc(target_logits, draft_logits, draft_tokens, u_bonus, temperature,
+                 log_weights_in, u_resample, ess_threshold, B, N, K, V, dtype, ws, out_tokens,
+                 log_weights_out, ess, ancestors, log_weight_increment,
+                 static_cast<cudaStream_t>(stream));
 }
 
 specdec_status specdec_verify_bf16(const void *target_logits, const void *draft_logits,
