@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--kernel-timing", choices=["on", "off"], default="on")
     ap.add_argument("--early-exit", choices=["on", "off"], default="on",
                     help="also time specdec_verify_early_exit on the same steps")
+    ap.add_argument("--topk", choices=["on", "off"], default="on",
+                    help="also time specdec_topk_exclude (k=60) over the target's draft rows")
     ap.add_argument("--smc", choices=["on", "off"], default="on",
                     help="also time specdec_smc_step (groups of 8 particles) on the same steps")
     return ap.parse_args()
@@ -391,6 +393,43 @@ def run_cuda(args):
                     "note": "one SMC-SD round over the same logits: statistics sweep, log "
                             "importance ratios and bonus draws, ESS and systematic resampling"}
 
+    # ---- LogitSpec candidates: top 60 of each target row, draft token left out
+    topk_line = None
+    if args.topk == "on":
+        kk = 60
+        nrows = B * K  # the target rows of the K draft positions
+        ridx = [torch.tensor([b * (K + 1) + i for b in range(B) for i in range(K)],
+                             dtype=torch.int64, device=dev)]
+        oidx = torch.empty((nrows, kk), dtype=torch.int32, device=dev)
+        oval = torch.empty((nrows, kk), dtype=torch.float32, device=dev)
+        ftk = L.specdec_topk_exclude
+
+        def tk(i):
+            b = bufs[i % ncopies]
+            return ftk(b["t"].data_ptr(), V, ridx[0].data_ptr(), nrows, V, dt_code,
+                       b["tok"].data_ptr(), kk, oidx.data_ptr(), oval.data_ptr(), sp)
+        for i in range(3):
+            if tk(i) != 0:
+                raise RuntimeError("specdec_topk_exclude failed")
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        k0 = torch.cuda.Event(enable_timing=True)
+        k1 = torch.cuda.Event(enable_timing=True)
+        k0.record(stream)
+        for i in range(args.steps):
+            tk(i)
+        k1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms_tk = sdist.max_over_ranks(k0.elapsed_time(k1), dev) / args.steps
+        row_bytes = V * (2 if w.dtype == "bf16" else 4)
+        topk_line = {"ms_per_call": ms_tk, "k": kk, "rows": nrows * world,
+                     "value": nrows * row_bytes * world / (ms_tk * 1e-3) / 1e9, "unit": "GB/s",
+                     "rows_per_s": nrows * world / (ms_tk * 1e-3),
+                     "note": "one read of each row counted; the candidate pass re-reads it "
+                             "from L2"}
+
     # ---- end to end through the host entry point (pinned buffers) ----------
     pin = {k: torch.from_numpy(np.ascontiguousarray(getattr(x, k))).pin_memory()
            for k in ("target", "draft", "tokens", "u_accept", "u_resample", "temperature")}
@@ -457,6 +496,8 @@ def run_cuda(args):
         line["early_exit"] = early
     if smc_line is not None:
         line["smc_step"] = smc_line
+    if topk_line is not None:
+        line["topk_exclude"] = topk_line
     line["e2e"] = {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                    "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
     line["clocks"] = sampler.summary()

@@ -210,6 +210,28 @@ specdec_status specdec_smc_step(const void *target_logits, const void *draft_log
                                 double *log_weights_out, double *ess, int32_t *ancestors,
                                 double *log_weight_increment, void *stream);
 
+/* Top-k candidates excluding one token (the LogitSpec page "LogitSpec:
+ * Accelerating Retrieval-based Speculative Decoding via Next Next Token
+ * Speculation", section 2, workflow step 2: once the next token x_{i+1} is
+ * known, the top k entries of the last logit row other than x_{i+1} are the
+ * candidates for the next-next token; the page uses k around 60).
+ * For output row r (0 <= r < rows), the input row is
+ *   logits + row_index[r] * row_stride   (row_index NULL: r * row_stride),
+ * V elements of dtype, any element alignment.  exclude[r] is the token to
+ * leave out (-1, or NULL for all rows, leaves none out).  Writes
+ * out_idx[r, 0..k-1] (int32) the token ids of the k largest logits, larger
+ * first and equal logits by ascending id, and, when out_val is not NULL,
+ * out_val[r, 0..k-1] (fp32) their logits (exactly).  Fewer than k tokens: the
+ * remaining entries are -1 / -inf.  A row holding a NaN is invalid: every
+ * entry -1 / NaN and SPECDEC_ERR_LOGITS in the device error word.
+ * Errors: SPECDEC_EINVAL for k outside [1, 256], row_stride < V, V < 1,
+ * rows < 0, null or misaligned pointers.  rows == 0 is a no-op.  Device
+ * memory, asynchronous on `stream`; no workspace. */
+specdec_status specdec_topk_exclude(const void *logits, long long row_stride,
+                                    const long long *row_index, int rows, int V,
+                                    specdec_dtype dtype, const int32_t *exclude, int k,
+                                    int32_t *out_idx, float *out_val, void *stream);
+
 /* End-to-end variant: every pointer is HOST memory (pinned memory makes the
  * copies asynchronous).  Copies the inputs to library-owned device buffers,
  * runs the verify step on `stream`, copies the outputs back and synchronises

@@ -38,6 +38,7 @@ _SIGS = {
     "specdec_verify_static": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P]),
     "specdec_smc_step": (_I, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_double, _I, _I, _I, _I, _I,
                               _P, _P, _P, _P, _P, _P]),
+    "specdec_topk_exclude": (_I, [_P, ctypes.c_longlong, _P, _I, _I, _I, _P, _I, _P, _P, _P]),
     "specdec_device_errors": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
     "specdec_release": (None, []),
     "specdec_status_string": (ctypes.c_char_p, [_I]),
@@ -190,6 +191,34 @@ def smc_step(target, draft, tokens, u_bonus, temperature, u_resample, N, ess_thr
                           out["increment"].data_ptr(), stream)
     _chk(st, "specdec_smc_step")
     return out
+
+
+def specdec_topk_exclude(logits, row_stride, row_index, rows, V, dtype, exclude, k, out_idx,
+                         out_val, stream) -> int:
+    return lib().specdec_topk_exclude(logits, row_stride, row_index, rows, V, dtype, exclude, k,
+                                      out_idx, out_val, stream)
+
+
+def topk_exclude(logits, k, exclude=None, row_index=None, stream=None):
+    """Top-k token ids (and logits) of each row of a [R, V] CUDA tensor (or of
+    the rows named by int64 ``row_index`` of a [*, V] tensor), leaving out
+    ``exclude[r]`` (int32, -1 = none).  Returns (idx [R', k] int32, val [R', k]
+    float32)."""
+    import torch
+    V = logits.shape[-1]
+    flat = logits.reshape(-1, V)
+    rows = flat.shape[0] if row_index is None else row_index.numel()
+    dev = logits.device
+    idx = torch.empty((rows, k), dtype=torch.int32, device=dev)
+    val = torch.empty((rows, k), dtype=torch.float32, device=dev)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    st = specdec_topk_exclude(flat.data_ptr(), flat.stride(0),
+                              None if row_index is None else row_index.data_ptr(), rows, V,
+                              _dtype_code(logits), None if exclude is None else exclude.data_ptr(),
+                              k, idx.data_ptr(), val.data_ptr(), stream)
+    _chk(st, "specdec_topk_exclude")
+    return idx, val
 
 
 def specdec_device_errors(stream=None) -> tuple:

@@ -1237,10 +1237,218 @@ __global__ void __launch_bounds__(NT) k_smc_resample(const double *__restrict__ 
 }
 
 // ---------------------------------------------------------------------------
+// kernel 4 (LogitSpec): top-k of a logit row, excluding one token
+// ---------------------------------------------------------------------------
+// The LogitSpec page ("LogitSpec: Accelerating Retrieval-based Speculative
+// Decoding via Next Next Token Speculation", section 2, workflow step 2):
+// after the next token x_{i+1} is known, the top k entries of the last logit
+// row other than x_{i+1} are the candidates for the next-next token.  Order:
+// larger logit first, equal logits by ascending token id; a row with a NaN is
+// invalid.  One CTA per row:
+//   1. one pass: each thread's running max of an order-preserving key of the
+//      logits (and a NaN check).  The k-th largest of the 512 thread maxima,
+//      tau0, is at most the row's k-th largest key (k distinct elements reach
+//      it), so every answer has key >= tau0;
+//   2. a second pass (from L2) appends every non-excluded element with
+//      key >= tau0 to a shared buffer (about k of them for real logits);
+//      a bitonic sort of (key, ~index) gives the order;
+//   3. when ties at the top overflow the buffer (e.g. a constant row), an
+//      exact radix select of the k-th key (8 bits per pass) and an
+//      index-ordered pick among the keys equal to it replace step 2.
+constexpr int kTopkThreads = 512;
+constexpr int kTopkMaxK = 256;
+constexpr int kTopkCap = 2048;  // candidate buffer (power of two)
+
+// order-preserving key: a larger logit has a larger key; never 0 for a
+// non-NaN value
+__device__ __forceinline__ uint32_t logit_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+template <typename T, typename F>
+__device__ __forceinline__ void row_foreach(const T *row, int V, F f) {
+  constexpr int VEC = Dt<T>::VEC;
+  const int head = row_head(row, (long long)V);
+  const int nvec = (V - head) / VEC;
+  if ((int)threadIdx.x < head) f((int)threadIdx.x, Dt<T>::load(row + threadIdx.x));
+  const uint4 *pv = reinterpret_cast<const uint4 *>(row + head);
+  for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
+    float x[VEC];
+    Dt<T>::unpack(__ldg(pv + i), x);
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) f(head + i * VEC + e, x[e]);
+  }
+  const int t0 = head + nvec * VEC;
+  if (t0 + (int)threadIdx.x < V) f(t0 + (int)threadIdx.x, Dt<T>::load(row + t0 + threadIdx.x));
+}
+
+// bitonic sort, descending, of n (a power of two, <= the block's reach) keys
+template <typename K>
+__device__ __forceinline__ void bitonic_desc(K *a, int n) {
+  for (int size = 2; size <= n; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      __syncthreads();
+      for (int i = threadIdx.x; i < n / 2; i += blockDim.x) {
+        const int lo = 2 * i - (i & (stride - 1));  // first of the pair
+        const int hi = lo + stride;
+        const bool desc = ((lo & size) == 0);
+        const K x = a[lo], y = a[hi];
+        if ((x < y) == desc) {
+          a[lo] = y;
+          a[hi] = x;
+        }
+      }
+    }
+  }
+  __syncthreads();
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kTopkThreads) k_topk_exclude(
+    const T *__restrict__ logits, long long row_stride, const long long *__restrict__ row_index,
+    int V, const int32_t *__restrict__ exclude, int k, int32_t *__restrict__ out_idx,
+    float *__restrict__ out_val) {
+  __shared__ unsigned long long cand[kTopkCap];  // (key << 32) | ~index
+  __shared__ uint32_t tmax[kTopkThreads];
+  __shared__ unsigned hist[256];
+  __shared__ int s_n, s_bad, s_rem, s_cnt[kTopkThreads / 32];
+  __shared__ uint32_t s_prefix;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const long long r = blockIdx.x;
+  const long long src = row_index ? row_index[r] : r;
+  const T *row = logits + src * row_stride;
+  const int ex0 = exclude ? exclude[r] : -1;
+  const int ex = (ex0 >= 0 && ex0 < V) ? ex0 : -1;
+  int32_t *oi = out_idx + r * k;
+  float *ov = out_val ? out_val + r * k : nullptr;
+  if (tid == 0) {
+    s_n = 0;
+    s_bad = 0;
+  }
+  // 1. thread maxima (and NaN check)
+  uint32_t mk = 0;
+  bool bad = false;
+  row_foreach(row, V, [&](int v, float x) {
+    bad |= isnan(x);
+    if (v != ex) mk = max(mk, logit_key(x));
+  });
+  tmax[tid] = mk;
+  if (__any_sync(FULL, bad) && lane == 0) s_bad = 1;
+  bitonic_desc(tmax, kTopkThreads);
+  if (s_bad) {  // invalid row
+    for (int i = tid; i < k; i += blockDim.x) {
+      oi[i] = -1;
+      if (ov) ov[i] = __int_as_float(0x7fc00000);
+    }
+    if (tid == 0) atomicOr(&g_error_flags, SPECDEC_ERR_LOGITS);
+    return;
+  }
+  const uint32_t tau0 = tmax[k - 1];  // 0 when fewer than k threads saw a value
+  // 2. candidates: every non-excluded key >= tau0
+  row_foreach(row, V, [&](int v, float x) {
+    const uint32_t key = logit_key(x);
+    if (v != ex && key >= tau0) {
+      const int pos = atomicAdd(&s_n, 1);
+      if (pos < kTopkCap)
+        cand[pos] = ((unsigned long long)key << 32) | (unsigned)(0xFFFFFFFFu - (unsigned)v);
+    }
+  });
+  __syncthreads();
+  int n = s_n;
+  if (n > kTopkCap) {
+    // 3. ties overflowed the buffer: exact k-th key by radix select
+    const int KB = sizeof(T) == 2 ? 16 : 32;  // bf16 keys live in the top 16 bits
+    uint32_t prefix = 0;
+    int rem = k;
+    for (int shift = 24; shift >= 32 - KB; shift -= 8) {
+      for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
+      __syncthreads();
+      const uint32_t hi_mask = (shift == 24) ? 0u : (0xFFFFFFFFu << (shift + 8));
+      row_foreach(row, V, [&](int v, float x) {
+        const uint32_t key = logit_key(x);
+        if (v != ex && (key & hi_mask) == (prefix & hi_mask)) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      });
+      __syncthreads();
+      if (tid == 0) {
+        int cum = 0, d = 255;
+        for (; d > 0; --d) {
+          if (cum + (int)hist[d] >= rem) break;
+          cum += (int)hist[d];
+        }
+        s_rem = rem - cum;
+        s_prefix = prefix | ((uint32_t)d << shift);
+      }
+      __syncthreads();
+      prefix = s_prefix;
+      rem = s_rem;
+      __syncthreads();
+    }
+    // tau = prefix (in the top KB bits); keys above it are k - rem elements,
+    // and the first `rem` (by index) of the keys equal to it complete the k
+    const uint32_t kmask = (KB == 32) ? 0xFFFFFFFFu : 0xFFFF0000u;
+    if (tid == 0) s_n = 0;
+    __syncthreads();
+    row_foreach(row, V, [&](int v, float x) {
+      const uint32_t key = logit_key(x) & kmask;
+      if (v != ex && key > prefix) {
+        const int pos = atomicAdd(&s_n, 1);
+        cand[pos] = ((unsigned long long)logit_key(x) << 32) |
+                    (unsigned)(0xFFFFFFFFu - (unsigned)v);
+      }
+    });
+    // equal keys in index order: contiguous elements per thread, block scan
+    const int E = (V + blockDim.x - 1) / blockDim.x;
+    const int e0 = min(tid * E, V), e1 = min(e0 + E, V);
+    int ce = 0;
+    for (int v = e0; v < e1; ++v)
+      if (v != ex && (logit_key(Dt<T>::load(row + v)) & kmask) == prefix) ++ce;
+    int incl = ce;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(FULL, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_cnt[warp] = incl;
+    __syncthreads();
+    int base = incl - ce;
+    for (int w = 0; w < warp; ++w) base += s_cnt[w];
+    const int ngt = k - rem;
+    for (int v = e0; v < e1 && base < rem; ++v) {
+      const float x = Dt<T>::load(row + v);
+      if (v != ex && (logit_key(x) & kmask) == prefix) {
+        cand[ngt + base] = ((unsigned long long)logit_key(x) << 32) |
+                           (unsigned)(0xFFFFFFFFu - (unsigned)v);
+        ++base;
+      }
+    }
+    __syncthreads();
+    n = k;
+  }
+  // sort the candidates (padded with 0 to a power of two) and write the first k
+  int np2 = 1;
+  while (np2 < n || np2 < k) np2 <<= 1;
+  for (int i = n + tid; i < np2; i += blockDim.x) cand[i] = 0ull;
+  bitonic_desc(cand, np2);
+  for (int i = tid; i < k; i += blockDim.x) {
+    const unsigned long long c = cand[i];
+    if (i < n && c != 0ull) {
+      const int v = (int)(0xFFFFFFFFu - (unsigned)(c & 0xFFFFFFFFull));
+      oi[i] = v;
+      if (ov) ov[i] = Dt<T>::load(row + v);
+    } else {
+      oi[i] = -1;
+      if (ov) ov[i] = -INFINITY;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-enum KernelId { KID_STATS = 0, KID_FINISH = 1, KID_SMC = 2, KID_COUNT = 3 };
-const char *kKernelNames[KID_COUNT] = {"k_row_stats", "k_finish", "k_smc_resample"};
+enum KernelId { KID_STATS = 0, KID_FINISH = 1, KID_SMC = 2, KID_TOPK = 3, KID_COUNT = 4 };
+const char *kKernelNames[KID_COUNT] = {"k_row_stats", "k_finish", "k_smc_resample",
+                                       "k_topk_exclude"};
 
 std::mutex g_mu;
 uint64_t g_launches[KID_COUNT];
@@ -1734,6 +1942,33 @@ specdec_status specdec_smc_step(const void *target_logits, const void *draft_log
                  log_weights_in, u_resample, ess_threshold, B, N, K, V, dtype, ws, out_tokens,
                  log_weights_out, ess, ancestors, log_weight_increment,
                  static_cast<cudaStream_t>(stream));
+}
+
+specdec_status specdec_topk_exclude(const void *logits, long long row_stride,
+                                    const long long *row_index, int rows, int V,
+                                    specdec_dtype dtype, const int32_t *exclude, int k,
+                                    int32_t *out_idx, float *out_val, void *stream) {
+  if (rows < 0 || V < 1 || k < 1 || k > kTopkMaxK || row_stride < V) return SPECDEC_EINVAL;
+  if (dtype != SPECDEC_F32 && dtype != SPECDEC_BF16) return SPECDEC_EINVAL;
+  if (rows == 0) return SPECDEC_OK;
+  if (!logits || !out_idx) return SPECDEC_EINVAL;
+  const uintptr_t es = dtype == SPECDEC_BF16 ? 2 : 4;
+  if (reinterpret_cast<uintptr_t>(logits) % es) return SPECDEC_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(exclude) | reinterpret_cast<uintptr_t>(out_idx) |
+       reinterpret_cast<uintptr_t>(out_val)) % 4 ||
+      reinterpret_cast<uintptr_t>(row_index) % 8)
+    return SPECDEC_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  LaunchTimer lt(KID_TOPK, st);
+  if (dtype == SPECDEC_BF16)
+    k_topk_exclude<__nv_bfloat16><<<(unsigned)rows, kTopkThreads, 0, st>>>(
+        static_cast<const __nv_bfloat16 *>(logits), row_stride, row_index, V, exclude, k, out_idx,
+        out_val);
+  else
+    k_topk_exclude<float><<<(unsigned)rows, kTopkThreads, 0, st>>>(
+        static_cast<const float *>(logits), row_stride, row_index, V, exclude, k, out_idx,
+        out_val);
+  return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ECUDA;
 }
 
 specdec_status specdec_verify_bf16(const void *target_logits, const void *draft_logits,

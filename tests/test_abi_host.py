@@ -41,8 +41,8 @@ def test_every_declared_symbol_is_exported(L):
 def test_status_strings_and_kernel_names(L):
     assert sd.status_string(sd.SPECDEC_OK) == "ok"
     assert "invalid" in sd.status_string(sd.SPECDEC_EINVAL)
-    assert sd.kernel_names() == ["k_row_stats", "k_finish", "k_smc_resample"]
-    assert len(sd.launch_counts()) == 3
+    assert sd.kernel_names() == ["k_row_stats", "k_finish", "k_smc_resample", "k_topk_exclude"]
+    assert len(sd.launch_counts()) == 4
 
 
 # fake, never-dereferenced addresses: validation must reject before any use
@@ -87,7 +87,7 @@ def test_workspace_size_is_monotone(L):
 def test_profile_api_without_launches(L):
     sd.profile_begin(4)
     res = sd.profile_end()
-    assert set(res) == {"k_row_stats", "k_finish", "k_smc_resample"}
+    assert set(res) == {"k_row_stats", "k_finish", "k_smc_resample", "k_topk_exclude"}
     assert all(c == 0 for _, c in res.values())
     assert L.specdec_profile_begin(0) == sd.SPECDEC_EINVAL
 
