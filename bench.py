@@ -56,6 +56,9 @@ def parse():
     ap.add_argument("--kernel-timing", choices=["on", "off"], default="on")
     ap.add_argument("--early-exit", choices=["on", "off"], default="on",
                     help="also time specdec_verify_early_exit on the same steps")
+    ap.add_argument("--chained", choices=["on", "off"], default="on",
+                    help="also time specdec_verify_chained (an intermediate tensor of the "
+                         "target's shape, the target logits as the final layer)")
     ap.add_argument("--topk", choices=["on", "off"], default="on",
                     help="also time specdec_topk_exclude (k=60) over the target's draft rows")
     ap.add_argument("--smc", choices=["on", "off"], default="on",
@@ -393,6 +396,46 @@ def run_cuda(args):
                     "note": "one SMC-SD round over the same logits: statistics sweep, log "
                             "importance ratios and bonus draws, ESS and systematic resampling"}
 
+    # ---- chained two-stage verify: final = the target, intermediate = its copy
+    # one position later in the rotation (distinct logits of the same shape) -----
+    chained_line = None
+    if args.chained == "on" and K <= 31:
+        u2 = torch.rand((B, K + 1), dtype=torch.float32, device=dev,
+                        generator=torch.Generator(device=dev).manual_seed(5))
+        o_tok = torch.empty((B, K + 1), dtype=torch.int32, device=dev)
+        o_em = torch.empty((B,), dtype=torch.int32, device=dev)
+        fch = L.specdec_verify_chained
+
+        def ch(i):
+            b = bufs[i % ncopies]
+            inter = bufs[(i + 1) % ncopies]["t"]
+            return fch(b["t"].data_ptr(), inter.data_ptr(), b["d"].data_ptr(), b["tok"].data_ptr(),
+                       b["ua"].data_ptr(), b["ur"].data_ptr(), u2.data_ptr(), b["ur"].data_ptr(),
+                       b["T"].data_ptr(), B, K, V, dt_code, o_tok.data_ptr(), o_em.data_ptr(),
+                       None, None, sp)
+        for i in range(3):
+            if ch(i) != 0:
+                raise RuntimeError("specdec_verify_chained failed")
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        c0 = torch.cuda.Event(enable_timing=True)
+        c1 = torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        for i in range(args.steps):
+            ch(i)
+        c1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms_ch = sdist.max_over_ranks(c0.elapsed_time(c1), dev) / args.steps
+        ch_bytes = (2 * (K + 1) + K) * V * (2 if w.dtype == "bf16" else 4) * B
+        chained_line = {"ms_per_step": ms_ch, "unit": "GB/s",
+                        "value": ch_bytes * world / (ms_ch * 1e-3) / 1e9,
+                        "bytes_per_step": ch_bytes * world,
+                        "note": "two sweeps: intermediate + draft (stage 1), then final + "
+                                "intermediate (stage 2); value counts one read of the three "
+                                "tensors"}
+
     # ---- LogitSpec candidates: top 60 of each target row, draft token left out
     topk_line = None
     if args.topk == "on":
@@ -498,6 +541,8 @@ def run_cuda(args):
         line["smc_step"] = smc_line
     if topk_line is not None:
         line["topk_exclude"] = topk_line
+    if chained_line is not None:
+        line["verify_chained"] = chained_line
     line["e2e"] = {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                    "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
     line["clocks"] = sampler.summary()

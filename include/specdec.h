@@ -232,6 +232,35 @@ specdec_status specdec_topk_exclude(const void *logits, long long row_stride,
                                     specdec_dtype dtype, const int32_t *exclude, int k,
                                     int32_t *out_idx, float *out_val, void *stream);
 
+/* Chained two-stage verify (the HiSpec page "HiSpec: Hierarchical Speculative
+ * Decoding for LLMs", section 2: a draft exit L_d, an intermediate verifier
+ * exit L_i and the final layer L_f; the intermediate rejects early without
+ * relaxing the final criterion; lossless by applying the speculative-decoding
+ * argument at both stages, L_d -> L_i -> L_f).
+ *   Stage 1 = specdec_verify with target intermediate_logits [B, K+1, V],
+ *     draft_logits [B, K, V], draft_tokens, u_accept1 [B, K], u_resample1 [B]:
+ *     n1 accepted tokens and one drawn token, m = n1 + 1 tokens s.
+ *   Stage 2 verifies s against final_logits [B, K+1, V] (row j scores s_j)
+ *     with the intermediate as proposal: s_j accepted iff
+ *     u_accept2[b, j] * q_i,j(s_j) < p_f,j(s_j), u_accept2 [B, K+1]; at the
+ *     first rejection n2 one token is drawn from max(0, p_f,n2 - q_i,n2)/Z
+ *     with u_resample2[b] (the inverse-CDF rule of specdec_verify); when all m
+ *     are accepted they are emitted and nothing is drawn (the final layer's row
+ *     after them is not an input).
+ * out_tokens [B, K+1]: the emitted tokens, then -1; out_num_emitted [B]: how
+ * many (n2 + 1, or m), -1 for an invalid sequence (any row of the three
+ * tensors, a draft token or the temperature, as in specdec_verify).
+ * stage1_tokens [B, K+1] / stage1_num_accepted [B] (nullable) receive stage 1's
+ * outputs.  K <= 31.  Device memory, asynchronous on `stream`, library-owned
+ * workspace.  Two statistics sweeps: both tensors of stage 1, then the final
+ * and intermediate tensors again for stage 2. */
+specdec_status specdec_verify_chained(
+    const void *final_logits, const void *intermediate_logits, const void *draft_logits,
+    const int32_t *draft_tokens, const float *u_accept1, const float *u_resample1,
+    const float *u_accept2, const float *u_resample2, const float *temperature, int B, int K,
+    int V, specdec_dtype dtype, int32_t *out_tokens, int32_t *out_num_emitted,
+    int32_t *stage1_tokens, int32_t *stage1_num_accepted, void *stream);
+
 /* End-to-end variant: every pointer is HOST memory (pinned memory makes the
  * copies asynchronous).  Copies the inputs to library-owned device buffers,
  * runs the verify step on `stream`, copies the outputs back and synchronises

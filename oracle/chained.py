@@ -47,8 +47,9 @@ def verify_chained(final, inter, draft, tokens, u_accept1, u_resample1, u_accept
     the margins of the stage-2 decisions (for counting boundary cases)."""
     from . import default as _default_oracle
     orc = orc or _default_oracle()
+    # (with diagnostics: the decision margins count stage-1 boundary cases)
     r1 = orc.verify(inter, draft, tokens, u_accept1, u_resample1, temperature, dtype=dtype,
-                    diag=False)
+                    diag=True)
     n1 = r1["num_accepted"]
     s = r1["out_tokens"]
     zf = _smc._widen(final, dtype)

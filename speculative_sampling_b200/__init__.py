@@ -39,6 +39,8 @@ _SIGS = {
     "specdec_smc_step": (_I, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_double, _I, _I, _I, _I, _I,
                               _P, _P, _P, _P, _P, _P]),
     "specdec_topk_exclude": (_I, [_P, ctypes.c_longlong, _P, _I, _I, _I, _P, _I, _P, _P, _P]),
+    "specdec_verify_chained": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P,
+                                    _P, _P, _P]),
     "specdec_device_errors": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
     "specdec_release": (None, []),
     "specdec_status_string": (ctypes.c_char_p, [_I]),
@@ -219,6 +221,43 @@ def topk_exclude(logits, k, exclude=None, row_index=None, stream=None):
                               k, idx.data_ptr(), val.data_ptr(), stream)
     _chk(st, "specdec_topk_exclude")
     return idx, val
+
+
+def specdec_verify_chained(final, inter, draft, tokens, u_accept1, u_resample1, u_accept2,
+                           u_resample2, temperature, B, K, V, dtype, out_tokens,
+                           out_num_emitted, stage1_tokens, stage1_num_accepted, stream) -> int:
+    return lib().specdec_verify_chained(final, inter, draft, tokens, u_accept1, u_resample1,
+                                        u_accept2, u_resample2, temperature, B, K, V, dtype,
+                                        out_tokens, out_num_emitted, stage1_tokens,
+                                        stage1_num_accepted, stream)
+
+
+def verify_chained(final, inter, draft, tokens, u_accept1, u_resample1, u_accept2, u_resample2,
+                   temperature, stream=None) -> dict:
+    """Chained two-stage verify on CUDA tensors (see specdec_verify_chained).
+    Returns a dict of CUDA int32 tensors: out_tokens [B,K+1], num_emitted [B],
+    stage1_tokens [B,K+1], stage1_n [B]."""
+    import torch
+    B, K1, V = final.shape
+    K = K1 - 1
+    dev = final.device
+    out = dict(out_tokens=torch.empty((B, K1), dtype=torch.int32, device=dev),
+               num_emitted=torch.empty((B,), dtype=torch.int32, device=dev),
+               stage1_tokens=torch.empty((B, K1), dtype=torch.int32, device=dev),
+               stage1_n=torch.empty((B,), dtype=torch.int32, device=dev))
+    _check_dev(final, inter, draft, tokens, u_accept1, u_resample1, u_accept2, u_resample2,
+               temperature)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    st = specdec_verify_chained(final.data_ptr(), inter.data_ptr(), draft.data_ptr(),
+                                tokens.data_ptr(), u_accept1.data_ptr(), u_resample1.data_ptr(),
+                                u_accept2.data_ptr(), u_resample2.data_ptr(),
+                                temperature.data_ptr(), B, K, V, _dtype_code(final),
+                                out["out_tokens"].data_ptr(), out["num_emitted"].data_ptr(),
+                                out["stage1_tokens"].data_ptr(), out["stage1_n"].data_ptr(),
+                                stream)
+    _chk(st, "specdec_verify_chained")
+    return out
 
 
 def specdec_device_errors(stream=None) -> tuple:

@@ -368,6 +368,8 @@ struct StatsGeom {
   int slots;        // CTA slots per row (>= CTAs that can share one row)
   int p0, np, rps;  // the window: first position, positions, rows per sequence
   const int *state; // per-sequence decision state, or null (every sequence)
+  int d_rows;       // rows per sequence of the draft tensor (K, or K+1 when it is an
+                    // intermediate verifier's logits)
 };
 __device__ __forceinline__ bool seq_active(const StatsGeom &g, long long b) {
   return g.state == nullptr || __ldcg(g.state + b) == kSeqActive;
@@ -397,7 +399,7 @@ struct RowCursor {
     constexpr int VEC = Dt<T>::VEC;
     const int pos = w < 2 * g.np ? g.p0 + (w >> 1) : g.K;
     const bool is_draft = w < 2 * g.np && (w & 1);
-    p = is_draft ? draft + (b * g.K + pos) * g.V : target + (b * (g.K + 1) + pos) * g.V;
+    p = is_draft ? draft + (b * g.d_rows + pos) * g.V : target + (b * (g.K + 1) + pos) * g.V;
     head = row_head(p, g.V);
     nvec = (g.V - head) / VEC;
     pv = reinterpret_cast<const uint4 *>(p + head);
@@ -724,13 +726,22 @@ __device__ __noinline__ int draw_exact64(const T *pt, const T *pd, long long V, 
 // every particle keeps its K draft tokens, draws its bonus token from p_K, and
 // gets the log importance ratio of its K tokens,
 // dlogw[b] = sum_i [log p_i(x_i) - log q_i(x_i)] in fp64 (-inf when invalid).
+//
+// Chained second stage (`len` set; the HiSpec page, section 2): sequence b
+// tests only its first m = len[b] + 1 tokens (the output of the first stage;
+// len[b] < 0: invalid there); when all m are accepted they are emitted with no
+// draw.  With `emit_count`, out_n holds the number of tokens emitted rather
+// than the number accepted.
 struct FinishWindow {
   int p0, np, bonus, rps;
   int decide_only;
   int *state;
   SeqInfo *info;
   double *dlogw;
+  const int32_t *len;
+  int emit_count;
 };
+constexpr int kChainAll = -3;  // chained stage: every tested token accepted
 
 template <typename T, int UW>
 __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
@@ -738,7 +749,7 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
     const int32_t *__restrict__ tokens, const float *__restrict__ u_accept,
     const float *__restrict__ u_resample, const float *__restrict__ temperature, int K,
     long long V, int tpr, long long tiles, long long G1, int slots, int nsr, int cpb,
-    FinishWindow fw, const Partial *__restrict__ part,
+    int d_rows, int tok_stride, FinishWindow fw, const Partial *__restrict__ part,
     ResPartial *__restrict__ rpart, unsigned *__restrict__ counters,
     int32_t *__restrict__ out_tokens, int32_t *__restrict__ out_n,
     float *__restrict__ dbg_row_max, double *__restrict__ dbg_row_sum,
@@ -747,8 +758,8 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
   constexpr long long CHV = 32LL * UW;                 // vectors per (warp-)chunk
   constexpr long long CH = CHV * VEC;                  // elements per chunk
   constexpr int EMAX = (int)((CH + 2 * VEC + NT - 1) / NT);  // rescan elements per thread
-  __shared__ float sM[65];
-  __shared__ double sS[65];
+  __shared__ float sM[66];
+  __shared__ double sS[66];
   __shared__ int s_n, s_last, s_mode, s_chunk, s_y, s_lastpos;
   __shared__ double s_base, s_t;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -766,13 +777,16 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
   bool x_ok = true;
   float zt_x = 0.f, zd_x = 0.f, u = 0.f;
   const int pos = fw.p0 + lane;  // the position lane `lane` of warp 0 tests
-  if (warp == 0 && lane < fw.np) {
-    x = __ldg(tokens + b * K + pos);
+  // positions of the window this sequence tests (chained stage: its first m)
+  const int len_b = fw.len ? __ldg(fw.len + b) : 0;
+  const int m_b = fw.len ? (len_b >= 0 ? len_b + 1 : 0) : fw.np;
+  if (warp == 0 && lane < m_b) {
+    x = __ldg(tokens + b * tok_stride + pos);
     x_ok = (x >= 0) && ((long long)x < V);
-    u = fw.dlogw ? 0.f : __ldg(u_accept + b * K + pos);  // (SMC-SD accepts no test)
+    u = fw.dlogw ? 0.f : __ldg(u_accept + b * tok_stride + pos);  // (SMC-SD accepts no test)
     if (x_ok) {
       zt_x = Dt<T>::load(target + (b * (K + 1) + pos) * V + x);
-      zd_x = Dt<T>::load(draft + (b * K + pos) * V + x);
+      zd_x = Dt<T>::load(draft + (b * d_rows + pos) * V + x);
     }
   }
   const float ures = __ldg(u_resample + b);
@@ -841,15 +855,15 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
       rows_ok = __all_sync(FULL, rows_ok) && !timed_out;
       bool acc_i = false;
       double p = 0.0, q = 0.0;
-      if (lane < fw.np && x_ok && rows_ok && t_ok) {
+      if (lane < m_b && x_ok && rows_ok && t_ok) {
         p = exp2(((double)zt_x - (double)sM[2 * lane]) * c64) / sS[2 * lane];
         q = exp2(((double)zd_x - (double)sM[2 * lane + 1]) * c64) / sS[2 * lane + 1];
         acc_i = (double)u * q < p;
       }
-      const unsigned bad_x = __ballot_sync(FULL, lane < fw.np && !x_ok);
-      const unsigned accm = __ballot_sync(FULL, lane < fw.np && acc_i);
-      const bool seq_ok = t_ok && rows_ok && bad_x == 0;
-      const unsigned kmask = (fw.np >= 32) ? FULL : ((1u << fw.np) - 1u);
+      const unsigned bad_x = __ballot_sync(FULL, lane < m_b && !x_ok);
+      const unsigned accm = __ballot_sync(FULL, lane < m_b && acc_i);
+      const bool seq_ok = t_ok && rows_ok && bad_x == 0 && !(fw.len && len_b < 0);
+      const unsigned kmask = (m_b >= 32) ? FULL : ((1u << m_b) - 1u);
       unsigned rej = ~accm & kmask;
       if (fw.dlogw) {
         // SMC-SD: keep every draft token; weight by the log ratio of the window
@@ -863,8 +877,9 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
         if (cb == 0 && lane == 0) fw.dlogw[b] = seq_ok ? lr : -INFINITY;
         rej = 0u;
       }
-      // the decision: rejected at n, all of K accepted (bonus), or still open
-      int nn = rej ? fw.p0 + __ffs(rej) - 1 : (fw.bonus ? K : kSeqActive);
+      // the decision: rejected at n, all of K accepted (bonus), still open,
+      // or (chained stage) all tested tokens accepted
+      int nn = rej ? fw.p0 + __ffs(rej) - 1 : (fw.bonus ? K : (fw.len ? kChainAll : kSeqActive));
       if (!seq_ok) nn = -1;
       if (lane == 0) s_n = nn;
       if (cb == 0) {
@@ -872,17 +887,19 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
         if (nn == -1) {
           for (int i = lane; i <= K; i += 32) ot[i] = -1;
         } else {
-          const int last = nn >= 0 ? nn : fw.p0 + fw.np;  // tokens accepted in the window
-          if (lane < fw.np && pos < last) ot[pos] = x;
-          if (nn >= 0)
-            for (int i = nn + 1 + lane; i <= K; i += 32) ot[i] = -1;
-          if (lane < fw.np && pos <= (nn >= 0 ? nn : K)) {
+          // tokens accepted in the window, then -1 after the decided position
+          const int last = nn >= 0 ? nn : (nn == kChainAll ? m_b : fw.p0 + fw.np);
+          if (lane < m_b && pos < last) ot[pos] = x;
+          const int tail = nn >= 0 ? nn + 1 : (nn == kChainAll ? m_b : K + 1);
+          for (int i = tail + lane; i <= K; i += 32) ot[i] = -1;
+          if (lane < m_b && pos <= (nn >= 0 ? nn : K)) {
             if (dbg_px) dbg_px[b * K + pos] = p;
             if (dbg_qx) dbg_qx[b * K + pos] = q;
           }
         }
         if (lane == 0) {
-          if (nn != kSeqActive) out_n[b] = nn;
+          if (nn == kChainAll) out_n[b] = m_b;
+          else if (nn != kSeqActive) out_n[b] = (fw.emit_count && nn >= 0) ? nn + 1 : nn;
           if (fw.state) fw.state[b] = nn;
           if (nn == -1) {
             unsigned f = 0;
@@ -892,12 +909,13 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
             atomicOr(&g_error_flags, f);
           }
           if (fw.decide_only && nn >= 0) {  // the drawn pair for the final pass
-            const int wt = nn == K ? 2 * fw.np : 2 * (nn - fw.p0);
+            const bool nb = nn == K && fw.bonus;  // drawn from the bonus row
+            const int wt = nb ? 2 * fw.np : 2 * (nn - fw.p0);
             SeqInfo si;
             si.Mt = sM[wt];
             si.St = sS[wt];
-            si.Md = nn == K ? 0.f : sM[wt + 1];
-            si.Sd = nn == K ? 1.0 : sS[wt + 1];
+            si.Md = nb ? 0.f : sM[wt + 1];
+            si.Sd = nb ? 1.0 : sS[wt + 1];
             fw.info[b] = si;
           }
         }
@@ -906,16 +924,20 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
     __syncthreads();
     n = s_n;
     if (n < 0 || fw.decide_only) return;  // invalid, still open, or not drawn in this pass
-    const int wt = n == K ? 2 * fw.np : 2 * (n - fw.p0);
+    // the bonus row only when the window holds it (a chained second stage
+    // rejecting its position K draws from that row's residual instead)
+    const bool nb = n == K && fw.bonus;
+    const int wt = nb ? 2 * fw.np : 2 * (n - fw.p0);
     Mt = sM[wt];
     St = sS[wt];
-    Md = n == K ? 0.f : sM[wt + 1];
-    Sd = n == K ? 1.0 : sS[wt + 1];
+    Md = nb ? 0.f : sM[wt + 1];
+    Sd = nb ? 1.0 : sS[wt + 1];
   }
 
   // ---- this CTA's chunk of the drawn row pair ----
   DrawRow d;
-  d.bonus = (n == K);
+  // (a sequence decided by an earlier pass at n == K was decided on the bonus)
+  d.bonus = (n == K) && (fw.bonus || st_b >= 0);
   d.Mt = Mt;
   d.Md = d.bonus ? 0.f : Md;
   if (d.bonus) Sd = 1.0;
@@ -924,7 +946,7 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
   d.lhi = (float)lam;
   d.llo = (float)(lam - (double)d.lhi);
   const T *pt = target + (b * (K + 1) + n) * V;
-  const T *pd = d.bonus ? pt : draft + (b * K + n) * V;
+  const T *pd = d.bonus ? pt : draft + (b * d_rows + n) * V;
 
   const int head = row_head(pt, V);
   const bool vec_ok = row_head(pd, V) == head;
@@ -1479,8 +1501,10 @@ struct Plan {
   int esize, vec, U, tpr, nsr, cpb;
   Sweep full;            // the whole batch, every row
   Sweep first, second;   // early exit: positions [0, P), then [P, K] with the bonus row
+  Sweep chain;           // chained second stage: positions [0, K] of two K+1-row tensors
   int slots_max;
-  size_t off_part, off_rpart, off_cnt, off_state, off_info, off_dlogw, total;
+  size_t off_part, off_rpart, off_cnt, off_state, off_info, off_dlogw, off_s1tok, off_s1n,
+      total;
 };
 
 int num_sms() {
@@ -1533,9 +1557,10 @@ bool make_plan(int B, int K, int V, specdec_dtype dtype, int sms, Plan &pl) {
   const int P = early_split(K);
   pl.first = make_sweep(B, 0, P, 0, pl.tpr, cap);
   pl.second = make_sweep(B, P, K - P, 1, pl.tpr, cap);
+  pl.chain = make_sweep(B, 0, K + 1, 0, pl.tpr, cap);
   pl.slots_max = pl.full.slots;
-  if (pl.first.slots > pl.slots_max) pl.slots_max = pl.first.slots;
-  if (pl.second.slots > pl.slots_max) pl.slots_max = pl.second.slots;
+  for (const Sweep *w : {&pl.first, &pl.second, &pl.chain})
+    if (w->slots > pl.slots_max) pl.slots_max = w->slots;
   // k_finish chunks: 32 lanes x kFinishUW vectors of the drawn row pair
   const long long nr = (nvec_max + 32LL * kFinishUW - 1) / (32LL * kFinishUW);
   pl.nsr = (int)(nr > 0 ? nr : 1);
@@ -1549,7 +1574,7 @@ bool make_plan(int B, int K, int V, specdec_dtype dtype, int sms, Plan &pl) {
   if ((long long)B * (K + 1) * (long long)V > (1LL << 56)) return false;
   size_t off = 0;
   pl.off_part = off;
-  off = align256(off + sizeof(Partial) * (size_t)rows * pl.slots_max * CW);
+  off = align256(off + sizeof(Partial) * (size_t)pl.chain.rows * pl.slots_max * CW);
   pl.off_rpart = off;
   off = align256(off + sizeof(ResPartial) * (size_t)B * pl.nsr);
   pl.off_cnt = off;
@@ -1560,6 +1585,10 @@ bool make_plan(int B, int K, int V, specdec_dtype dtype, int sms, Plan &pl) {
   off = align256(off + sizeof(SeqInfo) * (size_t)B);
   pl.off_dlogw = off;
   off = align256(off + sizeof(double) * (size_t)B);
+  pl.off_s1tok = off;
+  off = align256(off + sizeof(int32_t) * (size_t)B * (K + 1));
+  pl.off_s1n = off;
+  off = align256(off + sizeof(int32_t) * (size_t)B);
   pl.total = off > 0 ? off : 256;
   return true;
 }
@@ -1627,21 +1656,34 @@ struct LaunchTimer {
   }
 };
 
+// Options of one pass (see StatsGeom and FinishWindow).
+struct PassOpts {
+  int *state = nullptr;          // early exit: per-sequence decision state
+  SeqInfo *info = nullptr;       // early exit: drawn pairs decided by the first pass
+  bool decide_only = false;      // early exit, first pass
+  double *dlogw = nullptr;       // SMC-SD mode
+  const int32_t *len = nullptr;  // chained second stage: first-stage accepted counts
+  int d_rows = -1;               // rows per sequence of the draft tensor (default K)
+  int tok_stride = -1;           // row stride of tokens and u_accept (default K)
+  int emit_count = 0;            // out_n = tokens emitted instead of accepted
+};
+
 // One pass: a statistics sweep over `sw` (of the open sequences when `state`
 // is set and the pass is not the first), then k_finish over the same window
 // (programmatic dependent launch: its launch and gathers overlap the sweep).
 template <typename T>
 specdec_status launch_pass(const void *tg, const void *dr, const int32_t *tok, const float *ua,
                            const float *ur, const float *temp, int B, int K, int V,
-                           const Plan &pl, const Sweep &sw, int *state, SeqInfo *info,
-                           bool decide_only, char *ws, const specdec_debug *dbg,
-                           int32_t *out_tokens, int32_t *out_n, cudaStream_t st,
-                           double *dlogw = nullptr) {
+                           const Plan &pl, const Sweep &sw, const PassOpts &o, char *ws,
+                           const specdec_debug *dbg, int32_t *out_tokens, int32_t *out_n,
+                           cudaStream_t st) {
   const T *t = static_cast<const T *>(tg);
   const T *d = static_cast<const T *>(dr);
   Partial *part = reinterpret_cast<Partial *>(ws + pl.off_part);
   ResPartial *rp = reinterpret_cast<ResPartial *>(ws + pl.off_rpart);
   unsigned *cnt = reinterpret_cast<unsigned *>(ws + pl.off_cnt);
+  const int d_rows = o.d_rows > 0 ? o.d_rows : K;
+  const int tok_stride = o.tok_stride > 0 ? o.tok_stride : K;
   StatsGeom g;
   g.K = K;
   g.V = V;
@@ -1651,7 +1693,8 @@ specdec_status launch_pass(const void *tg, const void *dr, const int32_t *tok, c
   g.p0 = sw.p0;
   g.np = sw.np;
   g.rps = sw.rps;
-  g.state = decide_only ? nullptr : state;  // the first pass reads every sequence
+  g.state = o.decide_only ? nullptr : o.state;  // the first pass reads every sequence
+  g.d_rows = d_rows;
   cudaError_t e = cudaSuccess;
   {
     LaunchTimer lt(KID_STATS, st);
@@ -1667,22 +1710,25 @@ specdec_status launch_pass(const void *tg, const void *dr, const int32_t *tok, c
   {
     LaunchTimer lt(KID_FINISH, st);
     // a decide-only pass draws nothing: one CTA per sequence
-    const int cpb = decide_only ? pl.nsr : pl.cpb;
+    const int cpb = o.decide_only ? pl.nsr : pl.cpb;
     const unsigned g2 = (unsigned)((long long)B * ((pl.nsr + cpb - 1) / cpb));
     FinishWindow fw;
     fw.p0 = sw.p0;
     fw.np = sw.np;
     fw.bonus = sw.bonus;
     fw.rps = sw.rps;
-    fw.decide_only = decide_only ? 1 : 0;
-    fw.state = state;
-    fw.info = info;
-    fw.dlogw = dlogw;
+    fw.decide_only = o.decide_only ? 1 : 0;
+    fw.state = o.state;
+    fw.info = o.info;
+    fw.dlogw = o.dlogw;
+    fw.len = o.len;
+    fw.emit_count = o.emit_count;
     auto kern = k_finish<T, kFinishUW>;
     e = launch_pdl(kern, g2, NT, st, t, d, tok, ua, ur, temp, K, (long long)V, pl.tpr, sw.tiles,
-                   sw.G1, sw.slots, pl.nsr, cpb, fw, (const Partial *)part, rp, cnt, out_tokens,
-                   out_n, dbg ? dbg->row_max : nullptr, dbg ? dbg->row_sum : nullptr,
-                   dbg ? dbg->p_x : nullptr, dbg ? dbg->q_x : nullptr, dbg ? dbg->Z : nullptr);
+                   sw.G1, sw.slots, pl.nsr, cpb, d_rows, tok_stride, fw, (const Partial *)part, rp,
+                   cnt, out_tokens, out_n, dbg ? dbg->row_max : nullptr,
+                   dbg ? dbg->row_sum : nullptr, dbg ? dbg->p_x : nullptr,
+                   dbg ? dbg->q_x : nullptr, dbg ? dbg->Z : nullptr);
   }
   return e == cudaSuccess ? SPECDEC_OK : SPECDEC_ECUDA;
 }
@@ -1693,15 +1739,41 @@ specdec_status launch_all(const void *tg, const void *dr, const int32_t *tok, co
                           const Plan &pl, bool early_exit, char *ws, const specdec_debug *dbg,
                           int32_t *out_tokens, int32_t *out_n, cudaStream_t st) {
   if (!early_exit)
-    return launch_pass<T>(tg, dr, tok, ua, ur, temp, B, K, V, pl, pl.full, nullptr, nullptr,
-                          false, ws, dbg, out_tokens, out_n, st);
-  int *state = reinterpret_cast<int *>(ws + pl.off_state);
-  SeqInfo *info = reinterpret_cast<SeqInfo *>(ws + pl.off_info);
-  specdec_status s = launch_pass<T>(tg, dr, tok, ua, ur, temp, B, K, V, pl, pl.first, state,
-                                    info, true, ws, dbg, out_tokens, out_n, st);
+    return launch_pass<T>(tg, dr, tok, ua, ur, temp, B, K, V, pl, pl.full, PassOpts(), ws, dbg,
+                          out_tokens, out_n, st);
+  PassOpts o;
+  o.state = reinterpret_cast<int *>(ws + pl.off_state);
+  o.info = reinterpret_cast<SeqInfo *>(ws + pl.off_info);
+  o.decide_only = true;
+  specdec_status s = launch_pass<T>(tg, dr, tok, ua, ur, temp, B, K, V, pl, pl.first, o, ws, dbg,
+                                    out_tokens, out_n, st);
   if (s != SPECDEC_OK) return s;
-  return launch_pass<T>(tg, dr, tok, ua, ur, temp, B, K, V, pl, pl.second, state, info, false,
-                        ws, dbg, out_tokens, out_n, st);
+  o.decide_only = false;
+  return launch_pass<T>(tg, dr, tok, ua, ur, temp, B, K, V, pl, pl.second, o, ws, dbg,
+                        out_tokens, out_n, st);
+}
+
+// The chained two-stage verify: stage 1 is the verify with the intermediate
+// logits as target; stage 2 verifies its tokens against the final logits with
+// the intermediate as proposal (draft tensor of K+1 rows, tokens and uniforms
+// of K+1 per sequence, m = n1 + 1 tested positions, no bonus).
+template <typename T>
+specdec_status launch_chained(const void *fin, const void *inter, const void *dr,
+                              const int32_t *tok, const float *ua1, const float *ur1,
+                              const float *ua2, const float *ur2, const float *temp, int B,
+                              int K, int V, const Plan &pl, char *ws, int32_t *s1_tok,
+                              int32_t *s1_n, int32_t *out_tokens, int32_t *out_emitted,
+                              cudaStream_t st) {
+  specdec_status s = launch_pass<T>(inter, dr, tok, ua1, ur1, temp, B, K, V, pl, pl.full,
+                                    PassOpts(), ws, nullptr, s1_tok, s1_n, st);
+  if (s != SPECDEC_OK) return s;
+  PassOpts o;
+  o.len = s1_n;
+  o.d_rows = K + 1;
+  o.tok_stride = K + 1;
+  o.emit_count = 1;
+  return launch_pass<T>(fin, inter, s1_tok, ua2, ur2, temp, B, K, V, pl, pl.chain, o, ws,
+                        nullptr, out_tokens, out_emitted, st);
 }
 
 specdec_status check_args(const void *tg, const void *dr, const int32_t *tok, const float *ua,
@@ -1765,11 +1837,13 @@ specdec_status run_smc(const void *tg, const void *dr, const int32_t *tok, const
   char *w = static_cast<char *>(ws);
   int32_t *n_scratch = reinterpret_cast<int32_t *>(w + pl.off_state);
   double *inc = dlw ? dlw : reinterpret_cast<double *>(w + pl.off_dlogw);
+  PassOpts o;
+  o.dlogw = inc;
   specdec_status s = (dtype == SPECDEC_BF16)
-      ? launch_pass<__nv_bfloat16>(tg, dr, tok, nullptr, ub, temp, B, K, V, pl, pl.full,
-                                   nullptr, nullptr, false, w, nullptr, ot, n_scratch, st, inc)
-      : launch_pass<float>(tg, dr, tok, nullptr, ub, temp, B, K, V, pl, pl.full, nullptr,
-                           nullptr, false, w, nullptr, ot, n_scratch, st, inc);
+      ? launch_pass<__nv_bfloat16>(tg, dr, tok, nullptr, ub, temp, B, K, V, pl, pl.full, o, w,
+                                   nullptr, ot, n_scratch, st)
+      : launch_pass<float>(tg, dr, tok, nullptr, ub, temp, B, K, V, pl, pl.full, o, w, nullptr,
+                           ot, n_scratch, st);
   if (s != SPECDEC_OK) return s;
   LaunchTimer lt(KID_SMC, st);
   cudaLaunchConfig_t cfg = {};
@@ -1969,6 +2043,44 @@ specdec_status specdec_topk_exclude(const void *logits, long long row_stride,
         static_cast<const float *>(logits), row_stride, row_index, V, exclude, k, out_idx,
         out_val);
   return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ECUDA;
+}
+
+specdec_status specdec_verify_chained(
+    const void *final_logits, const void *intermediate_logits, const void *draft_logits,
+    const int32_t *draft_tokens, const float *u_accept1, const float *u_resample1,
+    const float *u_accept2, const float *u_resample2, const float *temperature, int B, int K,
+    int V, specdec_dtype dtype, int32_t *out_tokens, int32_t *out_num_emitted,
+    int32_t *stage1_tokens, int32_t *stage1_num_accepted, void *stream) {
+  if (K > 31) return SPECDEC_EINVAL;  // the second stage tests K+1 positions on one warp
+  specdec_status s = check_args(intermediate_logits, draft_logits, draft_tokens, u_accept1,
+                                u_resample1, temperature, B, K, V, dtype, out_tokens,
+                                out_num_emitted);
+  if (s != SPECDEC_OK || B == 0) return s;
+  const uintptr_t es = dtype == SPECDEC_BF16 ? 2 : 4;
+  if (!final_logits || !u_accept2 || !u_resample2 ||
+      reinterpret_cast<uintptr_t>(final_logits) % es ||
+      (reinterpret_cast<uintptr_t>(u_accept2) | reinterpret_cast<uintptr_t>(u_resample2) |
+       reinterpret_cast<uintptr_t>(stage1_tokens) |
+       reinterpret_cast<uintptr_t>(stage1_num_accepted)) % 4)
+    return SPECDEC_EINVAL;
+  Plan pl;
+  if (!make_plan(B, K, V, dtype, num_sms(), pl)) return SPECDEC_EINVAL;
+  void *ws = nullptr;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  s = ensure_buf(g_ws, pl.total, st, &ws);
+  if (s != SPECDEC_OK) return s;
+  char *w = static_cast<char *>(ws);
+  int32_t *s1t = stage1_tokens ? stage1_tokens : reinterpret_cast<int32_t *>(w + pl.off_s1tok);
+  int32_t *s1n =
+      stage1_num_accepted ? stage1_num_accepted : reinterpret_cast<int32_t *>(w + pl.off_s1n);
+  if (dtype == SPECDEC_BF16)
+    return launch_chained<__nv_bfloat16>(final_logits, intermediate_logits, draft_logits,
+                                         draft_tokens, u_accept1, u_resample1, u_accept2,
+                                         u_resample2, temperature, B, K, V, pl, w, s1t, s1n,
+                                         out_tokens, out_num_emitted, st);
+  return launch_chained<float>(final_logits, intermediate_logits, draft_logits, draft_tokens,
+                               u_accept1, u_resample1, u_accept2, u_resample2, temperature, B,
+                               K, V, pl, w, s1t, s1n, out_tokens, out_num_emitted, st);
 }
 
 specdec_status specdec_verify_bf16(const void *target_logits, const void *draft_logits,

@@ -1,0 +1,92 @@
+"""Chained two-stage verify (specdec_verify_chained) against its oracle
+(oracle/chained.py).  The intermediate exit's logits are the final ones plus
+seeded noise (rounded to the workload dtype); the draft exit's are the
+workload's draft.  Emitted tokens and counts are compared exactly except on
+boundary cases of either stage (a decision or draw within 1e-6 of its
+threshold, counted as in the verify tests)."""
+import numpy as np
+import pytest
+
+import gpu_helpers as H
+import oracle
+import speculative_sampling_b200 as sd
+from oracle import chained
+from speculative_sampling_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def _make(name, B=None, V=None, K=None, sigma_i=0.3, seed=11):
+    x = inputs.generate(name, B=B, V=V, K=K)
+    rng = np.random.default_rng(seed)
+    if x.dtype == "bf16":
+        zf = inputs.bf16_bits_to_f32(x.target)
+        inter = inputs.f32_to_bf16_bits((zf + sigma_i * rng.normal(size=zf.shape)).astype(np.float32))
+    else:
+        inter = (x.target + sigma_i * rng.normal(size=x.target.shape)).astype(np.float32)
+    u2 = (rng.integers(0, 2 ** 24, (x.B, x.K + 1)).astype(np.float32) * np.float32(2.0 ** -24))
+    ur2 = (rng.integers(0, 2 ** 24, x.B).astype(np.float32) * np.float32(2.0 ** -24))
+    return x, inter, u2, ur2
+
+
+def _gpu(x, inter, u2, ur2):
+    torch = H.require_cuda()
+    d = H.to_device(x)
+    dv = lambda a: (torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+                    .view(torch.bfloat16) if x.dtype == "bf16"
+                    else torch.from_numpy(np.ascontiguousarray(a)).cuda())
+    out = sd.verify_chained(d["target"], dv(inter), d["draft"], d["tokens"], d["u_accept"],
+                            d["u_resample"], torch.from_numpy(u2).cuda(),
+                            torch.from_numpy(ur2).cuda(), d["temperature"])
+    torch.cuda.synchronize()
+    return {k: v.cpu().numpy() for k, v in out.items()}
+
+
+def _check(x, inter, u2, ur2):
+    g = _gpu(x, inter, u2, ur2)
+    o = chained.verify_chained(x.target, inter, x.draft, x.tokens, x.u_accept, x.u_resample, u2,
+                               ur2, x.temperature, dtype=x.dtype)
+    bnd = oracle.boundary_mask(o["stage1"], H.BAND) | (o["margin2"] < H.BAND)
+    firm = ~bnd
+    assert np.array_equal(g["stage1_n"][firm], o["stage1_n"][firm])
+    assert np.array_equal(g["num_emitted"][firm], o["num_emitted"][firm])
+    assert np.array_equal(g["out_tokens"][firm], o["out_tokens"][firm])
+    assert int(np.sum(~firm)) <= max(1, int(1e-4 * x.B * (x.K + 1)))
+    return g, o
+
+
+@pytest.mark.parametrize("name,B,V,K", [
+    ("batched_b64_k5_v128256_bf16", None, None, None),
+    ("mix_b128_k4_v32000_bf16", 64, None, None),
+    ("large_b256_k8_v151936_f32", 24, 30011, None),
+    ("tiny_b1_k4_v1000_f32", None, None, None),
+    ("large_b256_k8_v151936_f32", 16, 4099, 1),
+])
+def test_chained_matches_oracle(name, B, V, K):
+    x, inter, u2, ur2 = _make(name, B=B, V=V, K=K)
+    g, o = _check(x, inter, u2, ur2)
+    # both stages do something on the larger batches
+    if x.B >= 16:
+        assert np.any(o["num_emitted"] < o["stage1_n"] + 1)
+
+
+def test_equal_intermediate_and_final_is_one_verify():
+    x, _, u2, ur2 = _make("mix_b128_k4_v32000_bf16", B=32, V=5003)
+    g, o = _check(x, x.target.copy(), u2, ur2)
+    v = H.oracle_verify(x)
+    firm = ~oracle.boundary_mask(v, H.BAND)
+    assert np.array_equal(g["num_emitted"][firm], v["num_accepted"][firm] + 1)
+
+
+def test_chained_invalid_inputs():
+    x, inter, u2, ur2 = _make("mix_b128_k4_v32000_bf16", B=8, V=3001)
+    tgt = x.target.copy()
+    nan = inputs.f32_to_bf16_bits(np.array([np.nan], np.float32))[0]
+    tgt[2, x.K, 9] = nan          # a final-layer row (the last one)
+    x.tokens[5, 0] = x.V          # a draft token
+    x.target = tgt
+    sd.specdec_device_errors(None)
+    g, o = _check(x, inter, u2, ur2)
+    assert g["num_emitted"][2] == -1 and g["num_emitted"][5] == -1
+    assert np.all(g["out_tokens"][[2, 5]] == -1)
+    sd.specdec_device_errors(None)
