@@ -183,13 +183,19 @@ __device__ __forceinline__ float warp_max_nan(float v) {
 // device error word and the kernel winds down (the producer first waits, again
 // bounded, for the copies it has in flight).
 
-constexpr int CW = 8;               // consumer warps
+#ifndef SPECDEC_SWEEP_WARPS
+#define SPECDEC_SWEEP_WARPS 8
+#endif
+#ifndef SPECDEC_SWEEP_CTAS_PER_SM
+#define SPECDEC_SWEEP_CTAS_PER_SM 3
+#endif
+constexpr int CW = SPECDEC_SWEEP_WARPS;  // consumer warps of a sweep CTA
 constexpr int NTC = CW * 32;        // consumer threads
 constexpr int NTS = NTC + 32;       // + one producer warp
 constexpr int NSTAGE = 3;           // depth of the shared-memory ring
 constexpr unsigned long long kWaitNs = 2000000000ull;  // a wait gives up after 2 s
 constexpr unsigned kSuspendNs = 20000;  // longest sleep of one try_wait round
-constexpr int kStatsCtasPerSm = 4;  // resident CTAs per SM the sweep is sized for
+constexpr int kStatsCtasPerSm = SPECDEC_SWEEP_CTAS_PER_SM;  // sweep CTAs per SM the grid is sized for
 constexpr int kFinishUW = 4;        // vectors per lane in a k_finish chunk
 constexpr int kFinishCtasPerSm = 4; // k_finish grids fit one wave of this many CTAs per SM
 
@@ -1268,7 +1274,7 @@ __global__ void __launch_bounds__(NT) k_smc_resample(const double *__restrict__ 
 // larger logit first, equal logits by ascending token id; a row with a NaN is
 // invalid.  One CTA per row:
 //   1. one pass: each thread's running max of an order-preserving key of the
-//      logits (and a NaN check).  The k-th largest of the 512 thread maxima,
+//      logits (and a NaN check).  The k-th largest of the 256 thread maxima,
 //      tau0, is at most the row's k-th largest key (k distinct elements reach
 //      it), so every answer has key >= tau0;
 //   2. a second pass (from L2) appends every non-excluded element with
@@ -1277,32 +1283,97 @@ __global__ void __launch_bounds__(NT) k_smc_resample(const double *__restrict__ 
 //   3. when ties at the top overflow the buffer (e.g. a constant row), an
 //      exact radix select of the k-th key (8 bits per pass) and an
 //      index-ordered pick among the keys equal to it replace step 2.
-constexpr int kTopkThreads = 512;
+constexpr int kTopkThreads = 256;
 constexpr int kTopkMaxK = 256;
 constexpr int kTopkCap = 2048;  // candidate buffer (power of two)
 
-// order-preserving key: a larger logit has a larger key; never 0 for a
-// non-NaN value
+// order-preserving key: a larger logit has a larger key, -0 and +0 the same
+// key (equal logits); never 0 for a non-NaN value
 __device__ __forceinline__ uint32_t logit_key(float f) {
-  const uint32_t u = __float_as_uint(f);
+  uint32_t u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0u;
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// f(index, logit) for every element of a row: scalar head, 16-byte vectors
+// (four independent loads in flight per thread), scalar tail
 template <typename T, typename F>
 __device__ __forceinline__ void row_foreach(const T *row, int V, F f) {
   constexpr int VEC = Dt<T>::VEC;
+  constexpr int UNR = 4;
   const int head = row_head(row, (long long)V);
   const int nvec = (V - head) / VEC;
   if ((int)threadIdx.x < head) f((int)threadIdx.x, Dt<T>::load(row + threadIdx.x));
   const uint4 *pv = reinterpret_cast<const uint4 *>(row + head);
-  for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
-    float x[VEC];
-    Dt<T>::unpack(__ldg(pv + i), x);
+  const int step = (int)blockDim.x;
+  for (int i0 = threadIdx.x; i0 < nvec; i0 += step * UNR) {
+    uint4 v[UNR];
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) f(head + i * VEC + e, x[e]);
+    for (int u = 0; u < UNR; ++u) {
+      const int i = i0 + u * step;
+      v[u] = i < nvec ? __ldg(pv + i) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < UNR; ++u) {
+      const int i = i0 + u * step;
+      if (i < nvec) {
+        float x[VEC];
+        Dt<T>::unpack(v[u], x);
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) f(head + i * VEC + e, x[e]);
+      }
+    }
   }
   const int t0 = head + nvec * VEC;
   if (t0 + (int)threadIdx.x < V) f(t0 + (int)threadIdx.x, Dt<T>::load(row + t0 + threadIdx.x));
+}
+
+// NaN-propagating max of the 8 (bf16) or 4 (fp32) logits of a 16-byte vector
+__device__ __forceinline__ uint32_t bf16x2_max_nan(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.NaN.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+template <typename T>
+__device__ __forceinline__ float vec_max_nan(const uint4 &v);
+template <>
+__device__ __forceinline__ float vec_max_nan<__nv_bfloat16>(const uint4 &v) {
+  const uint32_t m = bf16x2_max_nan(bf16x2_max_nan(v.x, v.y), bf16x2_max_nan(v.z, v.w));
+  return fmax_nan(__uint_as_float(m << 16), __uint_as_float(m & 0xFFFF0000u));
+}
+template <>
+__device__ __forceinline__ float vec_max_nan<float>(const uint4 &v) {
+  return fmax3_nan(fmax3_nan(__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z)),
+                   __uint_as_float(v.w), -INFINITY);
+}
+
+// The same walk as row_foreach, a whole 16-byte vector at a time:
+// fv(first element index, vector) for the body, fs(index, logit) for the
+// scalar head and tail.
+template <typename T, typename FV, typename FS>
+__device__ __forceinline__ void row_foreach_vec(const T *row, int V, FV fv, FS fs) {
+  constexpr int VEC = Dt<T>::VEC;
+  constexpr int UNR = 4;
+  const int head = row_head(row, (long long)V);
+  const int nvec = (V - head) / VEC;
+  if ((int)threadIdx.x < head) fs((int)threadIdx.x, Dt<T>::load(row + threadIdx.x));
+  const uint4 *pv = reinterpret_cast<const uint4 *>(row + head);
+  const int step = (int)blockDim.x;
+  for (int i0 = threadIdx.x; i0 < nvec; i0 += step * UNR) {
+    uint4 v[UNR];
+#pragma unroll
+    for (int u = 0; u < UNR; ++u) {
+      const int i = i0 + u * step;
+      v[u] = i < nvec ? __ldg(pv + i) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < UNR; ++u) {
+      const int i = i0 + u * step;
+      if (i < nvec) fv(head + i * VEC, v[u]);
+    }
+  }
+  const int t0 = head + nvec * VEC;
+  if (t0 + (int)threadIdx.x < V) fs(t0 + (int)threadIdx.x, Dt<T>::load(row + t0 + threadIdx.x));
 }
 
 // bitonic sort, descending, of n (a power of two, <= the block's reach) keys
@@ -1348,14 +1419,31 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk_exclude(
     s_n = 0;
     s_bad = 0;
   }
-  // 1. thread maxima (and NaN check)
-  uint32_t mk = 0;
-  bool bad = false;
-  row_foreach(row, V, [&](int v, float x) {
+  // 1. thread maxima (and NaN check): a packed max per vector; only the
+  // vector holding the excluded token is unpacked
+  constexpr int VEC = Dt<T>::VEC;
+  float mx = -INFINITY;
+  bool bad = false, seen = false;
+  auto scalar1 = [&](int v, float x) {
     bad |= isnan(x);
-    if (v != ex) mk = max(mk, logit_key(x));
-  });
-  tmax[tid] = mk;
+    if (v != ex) {
+      mx = fmax_nan(mx, x);
+      seen = true;
+    }
+  };
+  row_foreach_vec(row, V, [&](int v0, const uint4 &w) {
+    if (ex >= v0 && ex < v0 + VEC) {
+      float x[VEC];
+      Dt<T>::unpack(w, x);
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) scalar1(v0 + e, x[e]);
+    } else {
+      mx = fmax_nan(mx, vec_max_nan<T>(w));
+      seen = true;
+    }
+  }, scalar1);
+  bad |= isnan(mx);
+  tmax[tid] = (seen && !isnan(mx)) ? logit_key(mx) : 0u;
   if (__any_sync(FULL, bad) && lane == 0) s_bad = 1;
   bitonic_desc(tmax, kTopkThreads);
   if (s_bad) {  // invalid row
@@ -1367,15 +1455,24 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk_exclude(
     return;
   }
   const uint32_t tau0 = tmax[k - 1];  // 0 when fewer than k threads saw a value
-  // 2. candidates: every non-excluded key >= tau0
-  row_foreach(row, V, [&](int v, float x) {
+  // 2. candidates: every non-excluded key >= tau0 (a vector is unpacked only
+  // when its max reaches tau0)
+  auto scalar2 = [&](int v, float x) {
     const uint32_t key = logit_key(x);
     if (v != ex && key >= tau0) {
       const int pos = atomicAdd(&s_n, 1);
       if (pos < kTopkCap)
         cand[pos] = ((unsigned long long)key << 32) | (unsigned)(0xFFFFFFFFu - (unsigned)v);
     }
-  });
+  };
+  row_foreach_vec(row, V, [&](int v0, const uint4 &w) {
+    if (logit_key(vec_max_nan<T>(w)) >= tau0) {
+      float x[VEC];
+      Dt<T>::unpack(w, x);
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) scalar2(v0 + e, x[e]);
+    }
+  }, scalar2);
   __syncthreads();
   int n = s_n;
   if (n > kTopkCap) {

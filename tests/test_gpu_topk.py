@@ -60,6 +60,8 @@ def test_ties_constant_rows_and_inf():
     q[2, ::3] = -np.inf
     q[3] = -np.inf
     q[3, 100:105] = 2.0
+    q[4, ::2] = 0.0                                              # +0 and -0 are equal
+    q[4, 1::2] = -0.0
     ex = np.array([-1, 7, 3, 100, V - 1, 0])
     _check(q, "f32", 60, ex)
     _check(inputs.f32_to_bf16_bits(q), "bf16", 200, ex)
