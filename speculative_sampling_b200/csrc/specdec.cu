@@ -814,25 +814,43 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
     Sd = __ldcg(&si->Sd);
   } else {
     // ---- combine the V-split partials of every row of the window (fp64) ----
+    // Warp w takes rows w, w + NWARP, ...  The partials of a row are those of
+    // the CTAs of the statistics sweep that hold its tiles, in order, CW
+    // consumer warps each.  The first partial per lane of the warp's first two
+    // rows is loaded before either row is reduced, and longer lists (many CTAs
+    // per row, as at B = 1) are read four loads per lane at a time, so the L2
+    // round trips overlap; the order of the fp64 sums is unchanged.
+    auto row_slots = [&](int r) -> int {
+      const long long row = b * RW + r;
+      return (int)(tile_owner(row * tpr + tpr - 1, G1, tiles) - tile_owner(row * tpr, G1, tiles) +
+                   1) * CW;
+    };
+    Partial pre0, pre1;
+    pre0.m = pre1.m = -INFINITY;
+    pre0.s = pre1.s = 0.0;
+    if (warp < RW && lane < row_slots(warp)) pre0 = part[(b * RW + warp) * slots * CW + lane];
+    if (warp + NWARP < RW && lane < row_slots(warp + NWARP))
+      pre1 = part[(b * RW + warp + NWARP) * slots * CW + lane];
     for (int r = warp; r < RW; r += NWARP) {
       const long long row = b * RW + r;
       const Partial *P = part + row * slots * CW;
-      // partials of the CTAs of the statistics sweep that hold tiles of this
-      // row, in order, CW consumer warps each
-      const int nslot = (int)(tile_owner(row * tpr + tpr - 1, G1, tiles) -
-                              tile_owner(row * tpr, G1, tiles) + 1) * CW;
+      const int nslot = row_slots(r);
       // first 32 partials in registers (one load per lane), the rest streamed
-      Partial p0;
-      p0.m = -INFINITY;
-      p0.s = 0.0;
-      if (lane < nslot) p0 = P[lane];
+      Partial p0 = r == warp ? pre0 : pre1;
+      if (r >= warp + 2 * NWARP) {
+        p0.m = -INFINITY;
+        p0.s = 0.0;
+        if (lane < nslot) p0 = P[lane];
+      }
       float m = p0.m;
+#pragma unroll 4
       for (int s = lane + 32; s < nslot; s += 32) m = fmax_nan(m, P[s].m);
       m = warp_max_nan(m);
       double acc =
           (lane < nslot)
               ? ((p0.m == -INFINITY) ? p0.s : p0.s * exp2(((double)p0.m - (double)m) * c64))
               : 0.0;
+#pragma unroll 4
       for (int s = lane + 32; s < nslot; s += 32) {
         const Partial ps = P[s];
         acc += (ps.m == -INFINITY) ? ps.s : ps.s * exp2(((double)ps.m - (double)m) * c64);
