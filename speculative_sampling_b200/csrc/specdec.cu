@@ -458,6 +458,11 @@ __global__ void __launch_bounds__(NTS, kStatsCtasPerSm) k_row_stats(const T *__r
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
+  // Let the dependent k_finish grid launch now: its CTAs take the SM slots this
+  // grid's CTAs free as they finish and do their input gathers during the
+  // sweep's tail.  They read this kernel's results only after
+  // cudaGridDependencySynchronize, which waits for the whole grid to complete.
+  cudaTriggerProgrammaticLaunchCompletion();
   if (t0 >= t1) return;
 
   // The CTA's tiles [t0, t1) are walked as row segments: the tiles of one row
