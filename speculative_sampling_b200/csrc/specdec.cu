@@ -446,9 +446,6 @@ __global__ void __launch_bounds__(NTS, kStatsCtasPerSm) k_row_stats(const T *__r
   const long long t0 = tile_begin(blockIdx.x, G, g.tiles);
   const long long t1 = tile_begin(blockIdx.x + 1, G, g.tiles);
 
-  // the arrival tickets of k_finish (which runs after this kernel) start at 0
-  if (blockIdx.x == 0)
-    for (int i = threadIdx.x; i < B; i += blockDim.x) tickets[i] = 0u;
   if (threadIdx.x == 0) {
     for (int i = 0; i < NSTAGE; ++i) {
       mbar_init(&full[i], 1);
@@ -458,6 +455,14 @@ __global__ void __launch_bounds__(NTS, kStatsCtasPerSm) k_row_stats(const T *__r
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
+  // This grid is launched with programmatic dependent launch: up to here it may
+  // overlap the kernel before it on the stream (the previous call's k_finish,
+  // which reads this workspace, or whatever wrote the inputs).  From here on
+  // every such kernel has completed and its writes are visible.
+  cudaGridDependencySynchronize();
+  // the arrival tickets of k_finish (which runs after this kernel) start at 0
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < B; i += blockDim.x) tickets[i] = 0u;
   // Let the dependent k_finish grid launch now: its CTAs take the SM slots this
   // grid's CTAs free as they finish and do their input gathers during the
   // sweep's tail.  They read this kernel's results only after
@@ -779,6 +784,10 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
   const int cb = (int)((long long)blockIdx.x - b * ncb);  // this CTA: chunks cb*cpb ...
   const int R = 2 * K + 1;
   const int RW = fw.rps;  // rows of the window per sequence
+  // The kernel after this one on the stream (the next call's statistics sweep,
+  // or the SMC-SD resampling) may be placed as this grid's CTAs finish; it
+  // waits for this grid to complete before it touches anything this grid uses.
+  cudaTriggerProgrammaticLaunchCompletion();
 
   // ---- inputs of this call (independent of the statistics kernel) ----
   const float Tf = __ldg(temperature + b);
@@ -1739,12 +1748,12 @@ int resident_ctas(KernelT kernel, int threads, size_t smem) {
 // launch with programmatic stream serialisation: the kernel may be scheduled
 // while the previous one drains and waits for it with cudaGridDependencySynchronize
 template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, cudaStream_t st,
-                       Args... args) {
+cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem,
+                       cudaStream_t st, Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(block);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1823,8 +1832,7 @@ specdec_status launch_pass(const void *tg, const void *dr, const int32_t *tok, c
     // the sweep assumes its CTAs are co-resident only for speed, not for
     // progress: nothing waits on another CTA
     resident_ctas(kern, NTS, smem);
-    kern<<<(unsigned)sw.G1, NTS, smem, st>>>(t, d, temp, g, part, cnt, B);
-    e = cudaGetLastError();
+    e = launch_pdl(kern, (unsigned)sw.G1, NTS, smem, st, t, d, temp, g, part, cnt, B);
   }
   if (e != cudaSuccess) return SPECDEC_ECUDA;
   {
@@ -1844,7 +1852,7 @@ specdec_status launch_pass(const void *tg, const void *dr, const int32_t *tok, c
     fw.len = o.len;
     fw.emit_count = o.emit_count;
     auto kern = k_finish<T, kFinishUW>;
-    e = launch_pdl(kern, g2, NT, st, t, d, tok, ua, ur, temp, K, (long long)V, pl.tpr, sw.tiles,
+    e = launch_pdl(kern, g2, NT, 0, st, t, d, tok, ua, ur, temp, K, (long long)V, pl.tpr, sw.tiles,
                    sw.G1, sw.slots, pl.nsr, cpb, d_rows, tok_stride, fw, (const Partial *)part, rp,
                    cnt, out_tokens, out_n, dbg ? dbg->row_max : nullptr,
                    dbg ? dbg->row_sum : nullptr, dbg ? dbg->p_x : nullptr,
