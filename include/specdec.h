@@ -39,9 +39,17 @@
  * otherwise, pointers are DEVICE memory of the current CUDA device and the call
  * is asynchronous on `stream` (a cudaStream_t; NULL is the legacy default
  * stream): nothing is synchronised, results are valid once the stream reaches
- * the end of the call.  The logit pointers must be aligned to their element
- * size; 16-byte alignment of every row (V * element size a multiple of 16)
- * gives the fast vector path, other layouts take a slower scalar path.
+ * the end of the call.  The kernels are launched with programmatic dependent
+ * launch: a call's first kernel may be placed on the GPU while the kernel
+ * before it on the stream is still running, but it reads no input and writes
+ * nothing until that kernel has completed, so stream order holds for the
+ * caller's producers of the inputs.  The call's last kernel lets a following
+ * kernel launched with programmatic serialisation start early; such a kernel
+ * must call cudaGridDependencySynchronize() before it reads the outputs (as
+ * the programming model requires of it anyway).  The logit pointers must be
+ * aligned to their element size; 16-byte alignment of every row (V * element
+ * size a multiple of 16) gives the fast vector path, other layouts take a
+ * slower scalar path.
  *
  * Errors:
  *   SPECDEC_EINVAL  an argument is invalid (checked on the host before any
