@@ -1315,7 +1315,11 @@ __global__ void __launch_bounds__(NT) k_smc_resample(const double *__restrict__ 
 //   3. when ties at the top overflow the buffer (e.g. a constant row), an
 //      exact radix select of the k-th key (8 bits per pass) and an
 //      index-ordered pick among the keys equal to it replace step 2.
-constexpr int kTopkThreads = 256;
+// 512 threads per row, three CTAs per SM (all 320 rows of a B=64, K=5 batch
+// resident at once): more loads in flight than 256 threads, and a tighter
+// threshold (the k-th largest of 512 thread maxima)
+constexpr int kTopkThreads = 512;
+constexpr int kTopkCtasPerSm = 3;
 constexpr int kTopkMaxK = 256;
 constexpr int kTopkCap = 2048;  // candidate buffer (power of two)
 
@@ -1430,7 +1434,7 @@ __device__ __forceinline__ void bitonic_desc(K *a, int n) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kTopkThreads) k_topk_exclude(
+__global__ void __launch_bounds__(kTopkThreads, kTopkCtasPerSm) k_topk_exclude(
     const T *__restrict__ logits, long long row_stride, const long long *__restrict__ row_index,
     int V, const int32_t *__restrict__ exclude, int k, int32_t *__restrict__ out_idx,
     float *__restrict__ out_val) {
