@@ -432,8 +432,9 @@ def run_cuda(args):
         chained_line = {"ms_per_step": ms_ch, "unit": "GB/s",
                         "value": ch_bytes * world / (ms_ch * 1e-3) / 1e9,
                         "bytes_per_step": ch_bytes * world,
-                        "note": "two sweeps: intermediate + draft (stage 1), then final + "
-                                "intermediate (stage 2); value counts one read of the three "
+                        "note": "two sweeps: intermediate + draft (stage 1), then the final "
+                                "layer's rows (stage 2, with the intermediate's row statistics "
+                                "kept from stage 1); value counts one read of the three "
                                 "tensors"}
 
     # ---- LogitSpec candidates: top 60 of each target row, draft token left out

@@ -376,6 +376,7 @@ struct StatsGeom {
   const int *state; // per-sequence decision state, or null (every sequence)
   int d_rows;       // rows per sequence of the draft tensor (K, or K+1 when it is an
                     // intermediate verifier's logits)
+  int tonly;        // the window holds target rows p0 .. p0+np-1 only (rps = np)
 };
 __device__ __forceinline__ bool seq_active(const StatsGeom &g, long long b) {
   return g.state == nullptr || __ldcg(g.state + b) == kSeqActive;
@@ -403,8 +404,8 @@ struct RowCursor {
   int w, ti, head;
   __device__ __forceinline__ void point(const T *target, const T *draft, const StatsGeom &g) {
     constexpr int VEC = Dt<T>::VEC;
-    const int pos = w < 2 * g.np ? g.p0 + (w >> 1) : g.K;
-    const bool is_draft = w < 2 * g.np && (w & 1);
+    const int pos = g.tonly ? g.p0 + w : (w < 2 * g.np ? g.p0 + (w >> 1) : g.K);
+    const bool is_draft = !g.tonly && w < 2 * g.np && (w & 1);
     p = is_draft ? draft + (b * g.d_rows + pos) * g.V : target + (b * (g.K + 1) + pos) * g.V;
     head = row_head(p, g.V);
     nvec = (g.V - head) / VEC;
@@ -756,6 +757,14 @@ struct FinishWindow {
   double *dlogw;
   const int32_t *len;
   int emit_count;
+  // Row statistics kept across passes (the chained verify): with `save_t` set,
+  // the combined (max, sum) of every target row of the window is stored at
+  // save_t[b*(K+1) + position]; with `dstat` set, the sweep covered only the
+  // window's target rows (srows = np per sequence) and the draft rows' (max,
+  // sum) are read from dstat[b*(K+1) + position].
+  int srows;  // rows per sequence of the sweep's partials
+  Partial *save_t;
+  const Partial *dstat;
 };
 constexpr int kChainAll = -3;  // chained stage: every tested token accepted
 
@@ -834,19 +843,20 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
     // rows is loaded before either row is reduced, and longer lists (many CTAs
     // per row, as at B = 1) are read four loads per lane at a time, so the L2
     // round trips overlap; the order of the fp64 sums is unchanged.
+    const int RS = fw.srows;  // the sweep's rows per sequence (RW unless only targets)
     auto row_slots = [&](int r) -> int {
-      const long long row = b * RW + r;
+      const long long row = b * RS + r;
       return (int)(tile_owner(row * tpr + tpr - 1, G1, tiles) - tile_owner(row * tpr, G1, tiles) +
                    1) * CW;
     };
     Partial pre0, pre1;
     pre0.m = pre1.m = -INFINITY;
     pre0.s = pre1.s = 0.0;
-    if (warp < RW && lane < row_slots(warp)) pre0 = part[(b * RW + warp) * slots * CW + lane];
-    if (warp + NWARP < RW && lane < row_slots(warp + NWARP))
-      pre1 = part[(b * RW + warp + NWARP) * slots * CW + lane];
-    for (int r = warp; r < RW; r += NWARP) {
-      const long long row = b * RW + r;
+    if (warp < RS && lane < row_slots(warp)) pre0 = part[(b * RS + warp) * slots * CW + lane];
+    if (warp + NWARP < RS && lane < row_slots(warp + NWARP))
+      pre1 = part[(b * RS + warp + NWARP) * slots * CW + lane];
+    for (int r = warp; r < RS; r += NWARP) {
+      const long long row = b * RS + r;
       const Partial *P = part + row * slots * CW;
       const int nslot = row_slots(r);
       // first 32 partials in registers (one load per lane), the rest streamed
@@ -871,13 +881,30 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
       }
       acc = warp_sum(acc);
       if (lane == 0) {
-        sM[r] = m;
-        sS[r] = acc;
+        // the row's position and role, and its place in the window's order
+        const bool is_t = fw.dstat || !(r < 2 * fw.np && (r & 1));
+        const int rp = fw.dstat ? fw.p0 + r : (r < 2 * fw.np ? fw.p0 + (r >> 1) : K);
+        const int w = fw.dstat ? 2 * r : r;
+        sM[w] = m;
+        sS[w] = acc;
         // natural row index: target rows 0..K, then draft rows 0..K-1
-        const int rp = r < 2 * fw.np ? fw.p0 + (r >> 1) : K;
-        const int j = (r < 2 * fw.np && (r & 1)) ? K + 1 + rp : rp;
+        const int j = is_t ? rp : K + 1 + rp;
         if (cb == 0 && dbg_row_max) dbg_row_max[b * R + j] = m;
         if (cb == 0 && dbg_row_sum) dbg_row_sum[b * R + j] = acc;
+        if (cb == 0 && fw.save_t && is_t) {
+          Partial o;
+          o.s = acc;
+          o.m = m;
+          o.pad = 0;
+          fw.save_t[b * (K + 1) + rp] = o;
+        }
+      }
+    }
+    if (fw.dstat) {  // the draft rows' statistics, kept by an earlier pass
+      for (int i = threadIdx.x; i < fw.np; i += blockDim.x) {
+        const Partial *q = fw.dstat + b * (K + 1) + fw.p0 + i;
+        sM[2 * i + 1] = __ldcg(&q->m);
+        sS[2 * i + 1] = __ldcg(&q->s);
       }
     }
     __syncthreads();
@@ -1626,6 +1653,7 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // partition of tiles over CTAs.
 struct Sweep {
   int p0, np, bonus, rps;
+  int tonly;                  // target rows only (see StatsGeom)
   long long rows, tiles, G1;  // G1: CTAs of the statistics sweep
   int slots;                  // partial slots per row
 };
@@ -1634,10 +1662,11 @@ struct Plan {
   int esize, vec, U, tpr, nsr, cpb;
   Sweep full;            // the whole batch, every row
   Sweep first, second;   // early exit: positions [0, P), then [P, K] with the bonus row
-  Sweep chain;           // chained second stage: positions [0, K] of two K+1-row tensors
+  Sweep chain;           // chained second stage: the final layer's K+1 rows (the
+                         // intermediate's statistics are kept from the first stage)
   int slots_max;
   size_t off_part, off_rpart, off_cnt, off_state, off_info, off_dlogw, off_s1tok, off_s1n,
-      total;
+      off_rstat, total;
 };
 
 int num_sms() {
@@ -1646,12 +1675,29 @@ int num_sms() {
   return n > 0 ? n : 148;
 }
 
+Sweep make_sweep(int B, int p0, int np, int bonus, int tpr, long long cap);
+
+// A sweep over the target tensor's rows p0 .. p0+np-1 only.
+Sweep make_target_sweep(int B, int p0, int np, int tpr, long long cap) {
+  Sweep w = make_sweep(B, p0, np, 0, tpr, cap);  // (for the partition of np rows per sequence)
+  w.tonly = 1;
+  w.rps = np;
+  w.rows = (long long)B * np;
+  w.tiles = w.rows * tpr;
+  w.G1 = w.tiles < cap ? w.tiles : cap;
+  if (w.G1 < 1) w.G1 = 1;
+  const long long minr = w.tiles / w.G1;
+  w.slots = minr > 0 ? (int)((tpr - 1 + minr - 1) / minr + 1) : 1;
+  return w;
+}
+
 Sweep make_sweep(int B, int p0, int np, int bonus, int tpr, long long cap) {
   Sweep w;
   w.p0 = p0;
   w.np = np;
   w.bonus = bonus;
   w.rps = 2 * np + bonus;
+  w.tonly = 0;
   w.rows = (long long)B * w.rps;
   w.tiles = w.rows * tpr;
   w.G1 = w.tiles < cap ? w.tiles : cap;
@@ -1690,7 +1736,7 @@ bool make_plan(int B, int K, int V, specdec_dtype dtype, int sms, Plan &pl) {
   const int P = early_split(K);
   pl.first = make_sweep(B, 0, P, 0, pl.tpr, cap);
   pl.second = make_sweep(B, P, K - P, 1, pl.tpr, cap);
-  pl.chain = make_sweep(B, 0, K + 1, 0, pl.tpr, cap);
+  pl.chain = make_target_sweep(B, 0, K + 1, pl.tpr, cap);
   pl.slots_max = pl.full.slots;
   for (const Sweep *w : {&pl.first, &pl.second, &pl.chain})
     if (w->slots > pl.slots_max) pl.slots_max = w->slots;
@@ -1707,7 +1753,10 @@ bool make_plan(int B, int K, int V, specdec_dtype dtype, int sms, Plan &pl) {
   if ((long long)B * (K + 1) * (long long)V > (1LL << 56)) return false;
   size_t off = 0;
   pl.off_part = off;
-  off = align256(off + sizeof(Partial) * (size_t)pl.chain.rows * pl.slots_max * CW);
+  long long rows_max = pl.full.rows;
+  for (const Sweep *w : {&pl.first, &pl.second, &pl.chain})
+    if (w->rows > rows_max) rows_max = w->rows;
+  off = align256(off + sizeof(Partial) * (size_t)rows_max * pl.slots_max * CW);
   pl.off_rpart = off;
   off = align256(off + sizeof(ResPartial) * (size_t)B * pl.nsr);
   pl.off_cnt = off;
@@ -1722,6 +1771,8 @@ bool make_plan(int B, int K, int V, specdec_dtype dtype, int sms, Plan &pl) {
   off = align256(off + sizeof(int32_t) * (size_t)B * (K + 1));
   pl.off_s1n = off;
   off = align256(off + sizeof(int32_t) * (size_t)B);
+  pl.off_rstat = off;
+  off = align256(off + sizeof(Partial) * (size_t)B * (K + 1));
   pl.total = off > 0 ? off : 256;
   return true;
 }
@@ -1799,6 +1850,8 @@ struct PassOpts {
   int d_rows = -1;               // rows per sequence of the draft tensor (default K)
   int tok_stride = -1;           // row stride of tokens and u_accept (default K)
   int emit_count = 0;            // out_n = tokens emitted instead of accepted
+  Partial *save_t = nullptr;      // keep the target rows' statistics here (see FinishWindow)
+  const Partial *dstat = nullptr; // the draft rows' statistics from an earlier pass
 };
 
 // One pass: a statistics sweep over `sw` (of the open sequences when `state`
@@ -1828,6 +1881,7 @@ specdec_status launch_pass(const void *tg, const void *dr, const int32_t *tok, c
   g.rps = sw.rps;
   g.state = o.decide_only ? nullptr : o.state;  // the first pass reads every sequence
   g.d_rows = d_rows;
+  g.tonly = sw.tonly;
   cudaError_t e = cudaSuccess;
   {
     LaunchTimer lt(KID_STATS, st);
@@ -1848,7 +1902,10 @@ specdec_status launch_pass(const void *tg, const void *dr, const int32_t *tok, c
     fw.p0 = sw.p0;
     fw.np = sw.np;
     fw.bonus = sw.bonus;
-    fw.rps = sw.rps;
+    fw.rps = sw.tonly ? 2 * sw.np : sw.rps;  // the window: target and draft row per position
+    fw.srows = sw.rps;
+    fw.save_t = o.save_t;
+    fw.dstat = o.dstat;
     fw.decide_only = o.decide_only ? 1 : 0;
     fw.state = o.state;
     fw.info = o.info;
@@ -1896,14 +1953,18 @@ specdec_status launch_chained(const void *fin, const void *inter, const void *dr
                               int K, int V, const Plan &pl, char *ws, int32_t *s1_tok,
                               int32_t *s1_n, int32_t *out_tokens, int32_t *out_emitted,
                               cudaStream_t st) {
-  specdec_status s = launch_pass<T>(inter, dr, tok, ua1, ur1, temp, B, K, V, pl, pl.full,
-                                    PassOpts(), ws, nullptr, s1_tok, s1_n, st);
+  Partial *rstat = reinterpret_cast<Partial *>(ws + pl.off_rstat);
+  PassOpts o1;
+  o1.save_t = rstat;  // the intermediate rows' statistics, for the second stage
+  specdec_status s = launch_pass<T>(inter, dr, tok, ua1, ur1, temp, B, K, V, pl, pl.full, o1, ws,
+                                    nullptr, s1_tok, s1_n, st);
   if (s != SPECDEC_OK) return s;
   PassOpts o;
   o.len = s1_n;
   o.d_rows = K + 1;
   o.tok_stride = K + 1;
   o.emit_count = 1;
+  o.dstat = rstat;  // the second stage sweeps the final layer's rows only
   return launch_pass<T>(fin, inter, s1_tok, ua2, ur2, temp, B, K, V, pl, pl.chain, o, ws,
                         nullptr, out_tokens, out_emitted, st);
 }
