@@ -297,8 +297,8 @@ specdec_status specdec_device_errors(void *stream, uint32_t *flags);
  *   - Returns SPECDEC_ESIZE, launching nothing, when these sizes need more
  *     workspace than the array holds (compare specdec_workspace_bytes with
  *     SPECDEC_STATIC_SCRATCH_BYTES; B=64,K=5,V=128256 bf16 needs about
- *     0.3 MiB and fits up to B=867; K=8,V=151936 fp32 needs 2.2 MiB at B=256
- *     and fits up to B=460).
+ *     0.4 MiB and fits up to B=837; K=8,V=151936 fp32 needs 2.3 MiB at B=256
+ *     and fits up to B=449).
  *   - The first call on a device looks up the array's device address (once
  *     per device, with that device current); make that first call before any
  *     stream capture on that device.
