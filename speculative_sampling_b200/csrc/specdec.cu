@@ -6,21 +6,26 @@
 // "Speculative Decoding ... Llama 70B x2.4", section "The mathematical definition
 // from Leviathan et al.").  This file is the B200 implementation:
 //
-//   k_row_stats  one pass over every logit row (B*(2K+1) rows of V): split-V
-//                online softmax statistics (row max m, sum of 2^((z-m)*c)) with
-//                16-byte non-temporal-in-L1 vector loads, a per-thread running
-//                max, warp-shuffle and shared-memory combines.  It streams the
-//                whole input once and is the HBM-bound kernel of the step.
-//   k_accept     one warp per sequence: combines the V-split partials of each of
-//                the 2K+1 rows in fp64, gathers p_i(x_i), q_i(x_i), tests
-//                u*q < p on K lanes and finds the first rejection with
-//                __ballot_sync/__ffs; writes the accepted prefix.
-//   k_resample   streams only the selected row pair (target/draft row n, or the
-//                target's bonus row K), forms r(v) = max(0, p - q) on the fly,
-//                reduces it per V-chunk; the last CTA of each sequence (atomic
-//                ticket, no waiting) takes the fp64 exclusive prefix over
-//                chunks, finds the chunk holding u*Z and rescans that one chunk
-//                with a block-wide fp64 scan to emit the drawn token.
+//   k_row_stats     one pass over every logit row (B*(2K+1) rows of V): a
+//                   producer thread streams 16 KB tiles with TMA bulk copies
+//                   into a 3-stage shared-memory ring (full/empty mbarriers,
+//                   every wait bounded); 8 consumer warps fold them into
+//                   split-V softmax statistics (row max m, sum of 2^((z-m)*c))
+//                   and write one partial per warp and row segment.  It streams
+//                   the whole input once and is the HBM-bound kernel.
+//   k_finish        per sequence, on several CTAs: combines the partials of the
+//                   2K+1 rows in fp64, gathers p_i(x_i), q_i(x_i), tests
+//                   u*q < p on K lanes (__ballot_sync/__ffs), writes the
+//                   accepted prefix; sums r(v) = max(0, p - q) (or the bonus
+//                   row) over its chunks of the drawn row pair; the last CTA of
+//                   the sequence (atomic ticket, no waiting) finds the chunk
+//                   holding u*Z from the fp64 chunk prefix and rescans it.
+//   k_smc_resample  SMC-SD: log-weights, effective sample size and systematic
+//                   resampling per group of particles.
+//   k_topk_exclude  top-k token ids of a row leaving one token out.
+// The verify kernels are launched with programmatic dependent launch: each
+// signals its dependents at its start and waits for its predecessor
+// (cudaGridDependencySynchronize) only where it first needs its results.
 //
 // Arithmetic: logits are widened exactly to fp32.  Exponentials are
 // 2^((z - m) * c) with c = log2(e)/T carried as an fp32 pair (hi + lo, with
@@ -2364,8 +2369,8 @@ specdec_status specdec_verify_static(const void *target_logits, const void *draf
   s = static_scratch_address(&scratch);
   if (s != SPECDEC_OK) return s;
   // Nothing in the scratch has to start at zero: every record the kernels read
-  // (V-split partials, per-sequence selection, chunk sums, the arrival counters
-  // that k_accept resets) is written earlier in the same call.
+  // (V-split partials, decisions, chunk sums, the arrival tickets that
+  // k_row_stats zeroes) is written earlier in the same call.
   return run(target_logits, draft_logits, draft_tokens, u_accept, u_resample, temperature, B, K,
              V, dtype, scratch, (size_t)SPECDEC_STATIC_SCRATCH_BYTES, nullptr, out_tokens,
              out_num_accepted, static_cast<cudaStream_t>(stream));
