@@ -11,7 +11,7 @@ inaccurate ones early, without relaxing the final acceptance criterion; the
 output is lossless because the lossless speculative-decoding argument is
 applied in turn at both stages (L_d -> L_i -> L_f).
 
-Readings where the page is silent (stated in the design notes):
+Readings taken where the page is silent:
   * stage 1 is the verify step with target L_i and draft L_d: the accepted
     prefix x_0..x_{n1-1} and the token y1 drawn at n1 (from max(0, p_i - q_d),
     or from L_i's row K when every draft token is accepted);
@@ -43,8 +43,12 @@ def verify_chained(final, inter, draft, tokens, u_accept1, u_resample1, u_accept
                    temperature, dtype: str = "f32", orc=None) -> dict:
     """final, inter [B, K+1, V]; draft [B, K, V]; tokens [B, K]; u_accept1 [B, K];
     u_resample1 [B]; u_accept2 [B, K+1]; u_resample2 [B]; temperature [B].
-    Returns out_tokens [B, K+1], num_emitted [B], stage1 tokens and n1, and
-    the margins of the stage-2 decisions (for counting boundary cases)."""
+    Returns out_tokens [B, K+1], num_emitted [B], stage1 tokens and n1, the
+    margins of the stage-2 decisions (for counting boundary cases), and the
+    stage-2 diagnostics: the final layer's row maxima and normalisers
+    sum_v exp((z_v - max)/T) [B, K+1], p_f,j(s_j) and q_i,j(s_j) for the tested
+    positions j (NaN elsewhere) [B, K+1], and the mass Z2 = sum max(0, p_f - q_i)
+    of the stage-2 residual draw (NaN when nothing is drawn) [B]."""
     from . import default as _default_oracle
     orc = orc or _default_oracle()
     # (with diagnostics: the decision margins count stage-1 boundary cases)
@@ -61,16 +65,26 @@ def verify_chained(final, inter, draft, tokens, u_accept1, u_resample1, u_accept
     out = np.full((B, K1), -1, np.int64)
     emitted = np.full(B, -1, np.int64)
     margin = np.full(B, np.inf)
+    f_max = np.full((B, K1), np.nan)
+    f_sum = np.full((B, K1), np.nan)
+    p2 = np.full((B, K1), np.nan)
+    q2 = np.full((B, K1), np.nan)
+    z2 = np.full(B, np.nan)
     for b in range(B):
         if n1[b] < 0 or not all(_smc._row_ok(zf[b, j]) for j in range(K1)):
             continue
         T = Tv[b]
+        for j in range(K1):  # diagnostics of the final layer's rows
+            f_max[b, j] = np.max(zf[b, j])
+            f_sum[b, j] = np.sum(np.exp((zf[b, j] - f_max[b, j]) / T))
         m = int(n1[b]) + 1
         n2 = m
         for j in range(m):
             p = _softmax(zf[b, j], T)
             q = _softmax(zi[b, j], T)
             tok = int(s[b, j])
+            p2[b, j] = p[tok]
+            q2[b, j] = q[tok]
             a = p[tok] / q[tok] if q[tok] > 0 else np.inf
             if a < 1.0:
                 margin[b] = min(margin[b], abs(u2[b, j] - a))
@@ -82,6 +96,7 @@ def verify_chained(final, inter, draft, tokens, u_accept1, u_resample1, u_accept
             p = _softmax(zf[b, n2], T)
             q = _softmax(zi[b, n2], T)
             r = np.maximum(0.0, p - q)
+            z2[b] = np.sum(r)
             if not (np.sum(r) > 0.0):
                 r = p
             y = _smc.inverse_cdf(r, ur2[b])
@@ -94,4 +109,5 @@ def verify_chained(final, inter, draft, tokens, u_accept1, u_resample1, u_accept
         else:
             emitted[b] = m
     return {"out_tokens": out, "num_emitted": emitted, "stage1_tokens": s, "stage1_n": n1,
-            "stage1": r1, "margin2": margin}
+            "stage1": r1, "margin2": margin, "row_max_f": f_max, "row_sum_f": f_sum,
+            "p2_x": p2, "q2_x": q2, "Z2": z2}

@@ -22,7 +22,7 @@
  * Temperature (the blog's vLLM example, temperature=0.7, and trade-off 4
  * "high temperature ruins the gain") enters as softmax(z / T) on BOTH models.
  *
- * Readings where the pages are silent (each one is listed in the design notes):
+ * Readings taken where the pages are silent:
  *   - accept iff  u * q(x) < p(x)  with u in [0,1)   (same as u < p/q; q = 0 and
  *     p > 0 accepts; p = q = 0 rejects);
  *   - row i of the target pairs with row i of the draft and token x_i; target

@@ -13,7 +13,7 @@ re-weighted by the ratio of target to draft probabilities; when the effective
 sample size falls below a threshold, low-weight particles are dropped and
 high-weight ones copied.
 
-Readings where the page is silent (each stated in the design notes):
+Readings taken where the page is silent:
   * temperature softmax on both models, as in the verify step;
   * the weight of a particle is the importance ratio of its K new tokens,
     log w += sum_i [log p_i(x_i) - log q_i(x_i)] (the tokens were drawn from q,

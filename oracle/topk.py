@@ -10,7 +10,7 @@ the top k entries of the last logit row, excluding x_{i+1}, are taken as the
 candidates for the next-next token (the page reports the true next-next token
 inside the top 60 in more than half of the decoding steps).
 
-Readings where the page is silent (stated in the design notes):
+Readings taken where the page is silent:
   * order: by logit, largest first; equal logits by ascending token id (so the
     result is unique);
   * the excluded token is never returned; exclude = -1 excludes nothing;

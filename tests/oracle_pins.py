@@ -355,6 +355,58 @@ def check_thread_invariance(orc):
         assert np.array_equal(r1[k], r8[k], equal_nan=True), k
 
 
+def check_zero_residual_draws_from_target_row(orc):
+    """Z = 0 after a rejection (reachable only through rounding) draws from p_n.
+
+    Draft row 0 equals target row 0, so p_0 = q_0 exactly; the draft token's
+    logit is so low that p_0(x) = q_0(x) = 0 in fp64, so u*q < p fails and the
+    walk rejects at n = 0.  The residual max(0, p_0 - q_0) is then zero
+    everywhere.  The reading for this case draws from p_0 itself; the result must
+    be numpy's inverse CDF of p_0 (cumsum + searchsorted, side='right'), not a
+    draw from another row, and not -1."""
+    T = 1.0
+    z0 = np.array([0.3, -0.2, 1.1, 0.0, -0.7, -1000.0], np.float32)
+    zt = np.stack([z0, np.array([2.0, -1.0, 0.5, 0.1, 0.0, 1.5], np.float32),
+                   np.array([-0.5, 0.9, 0.2, 3.0, -2.0, 0.4], np.float32)])
+    zd = np.stack([z0, zt[1] + np.float32(0.5)])
+    us = [0.0, 0.1, 0.35, 0.6, 0.9, 0.999]
+    res = _call(orc, zt, zd, [[5, 0]] * len(us), [[0.5, 0.5]] * len(us), us, T)
+    p0 = softmax64(zt[0], T)
+    assert p0[5] == 0.0  # the draft token has probability 0 in both rows
+    cdf = np.cumsum(p0)
+    want = np.searchsorted(cdf, np.asarray(us, np.float64) * cdf[-1], side="right")
+    assert np.all(res["num_accepted"] == 0)
+    assert np.array_equal(res["out_tokens"][:, 0], want), (res["out_tokens"][:, 0], want)
+    assert np.all(res["out_tokens"][:, 1:] == -1)
+    assert np.allclose(res["Z"], 1.0, rtol=0, atol=1e-12)  # mass of p_0
+    assert np.all(res["margin_sample"] == 0.0)             # counted as a boundary draw
+
+
+def check_no_cell_reached_takes_last_positive(orc):
+    """When no running sum exceeds u*Z (u = 1 reaches this exactly: t equals the
+    total), the draw is the largest index with positive weight: the limit of the
+    inverse CDF as u -> 1.  Checked on a bonus row and on a residual whose last
+    entries have zero weight, against the draw at the largest fp32 uniform below
+    1 (whose cell is the same last positive one)."""
+    T = 1.0
+    V = 8
+    # bonus draw: draft = target, every token accepted; p_1 is zero on 6, 7
+    zb = np.array([[0.1, 0.4, -0.3, 0.8, 0.0, 0.2, -np.inf, -np.inf],
+                   [0.5, -0.1, 0.3, 0.0, 0.9, 0.2, -np.inf, -np.inf]], np.float32)
+    u_top = float(np.float32(1.0) - np.float32(2.0 ** -24))
+    res = _call(orc, zb, zb[:1], [[3], [3]], [[0.5], [0.5]], [1.0, u_top], T)
+    assert np.all(res["num_accepted"] == 1)
+    assert list(res["out_tokens"][:, 1]) == [5, 5], res["out_tokens"]
+    # residual draw: p - q is positive only on tokens 0 and 2 (so index 2 is last)
+    pt = np.array([0.30, 0.05, 0.25, 0.10, 0.10, 0.10, 0.05, 0.05])
+    pd = np.array([0.10, 0.10, 0.10, 0.15, 0.15, 0.15, 0.125, 0.125])
+    zt = np.log(np.stack([pt, np.full(V, 1.0 / V)])).astype(np.float32)
+    zd = np.log(pd[None]).astype(np.float32)
+    res = _call(orc, zt, zd, [[6], [6]], [[0.99], [0.99]], [1.0, u_top], T)
+    assert np.all(res["num_accepted"] == 0)
+    assert list(res["out_tokens"][:, 0]) == [2, 2], res["out_tokens"]
+
+
 ALL_CHECKS = [
     check_hand_cases,
     check_law_suite,
@@ -366,5 +418,7 @@ ALL_CHECKS = [
     check_invalid_inputs,
     check_thread_invariance,
     check_diagnostics_do_not_change_results,
+    check_zero_residual_draws_from_target_row,
+    check_no_cell_reached_takes_last_positive,
     check_chi_square,
 ]

@@ -124,3 +124,26 @@ def test_invalid_final_row_invalidates():
                                np.zeros((3, x.K + 1), np.float32), x.u_resample, x.temperature)
     assert r["num_emitted"][1] == -1 and np.all(r["out_tokens"][1] == -1)
     assert r["num_emitted"][0] >= 1
+
+
+def test_stage2_diagnostics_match_the_verify_oracle():
+    """With the intermediate layer equal to the final one, the second stage's
+    row statistics are those the C verify oracle computes for the same rows,
+    every tested token has p_f = q_i (so it is accepted), and no residual is
+    drawn."""
+    from speculative_sampling_b200 import inputs
+    x = inputs.generate("mix_b128_k4_v32000_bf16", B=12, V=1999)
+    rng = np.random.default_rng(7)
+    u2 = rng.random((12, x.K + 1)).astype(np.float32)
+    r = chained.verify_chained(x.target, x.target, x.draft, x.tokens, x.u_accept, x.u_resample,
+                               u2, x.u_resample, x.temperature, dtype="bf16")
+    v = oracle.verify(x.target, x.draft, x.tokens, x.u_accept, x.u_resample, x.temperature,
+                      dtype="bf16", diag=True)
+    ok = v["num_accepted"] >= 0
+    K1 = x.K + 1
+    assert np.array_equal(r["row_max_f"][ok], v["row_max"][ok, :K1])
+    assert np.allclose(r["row_sum_f"][ok], v["row_sum"][ok, :K1], rtol=1e-12, atol=0)
+    tested = np.isfinite(r["p2_x"])
+    assert np.array_equal(tested[ok].sum(axis=1), v["num_accepted"][ok] + 1)
+    assert np.allclose(r["p2_x"][tested], r["q2_x"][tested], rtol=1e-12, atol=0)
+    assert np.all(np.isnan(r["Z2"]))

@@ -28,6 +28,14 @@ MUTANTS = {
                                      "const double t = (double)j->u_resample[b];"),
     "no_stop_at_first_rejection": ("      n = i;\n      break;", "      n = i;\n      continue;"),
     "tail_not_padded": ("for (int i = n + 1; i <= K; ++i) out[i] = -1;", ""),
+    "zero_residual_draws_from_bonus_row": (
+        "r[v] = prob(j->target, j->dtype, toff[n], v, M[n], S[n], T);",
+        "r[v] = prob(j->target, j->dtype, toff[K], v, M[K], S[K], T);"),
+    "zero_residual_not_handled": ("if (Z == 0.0) { /* only reachable", "if (0) { /* only reachable"),
+    "no_cell_reached_takes_last_index": ("      if (r[v] > 0.0) {\n        y = v;",
+                                         "      if (1) {\n        y = v;"),
+    "no_cell_reached_takes_first_positive": ("for (int64_t v = V - 1; v >= 0; --v)\n      if (r[v] > 0.0)",
+                                             "for (int64_t v = 0; v < V; ++v)\n      if (r[v] > 0.0)"),
     "bf16_misread": ("uint32_t bits = (uint32_t)((const uint16_t *)base)[idx] << 16;",
                      "uint32_t bits = (uint32_t)((const uint16_t *)base)[idx] << 15;"),
 }
