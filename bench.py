@@ -76,9 +76,12 @@ def measured_peaks():
 
 
 def stored_traffic():
-    """dram bytes per launch of k_row_stats from the committed ncu capture,
-    valid only while the kernel source is unchanged since the capture."""
-    p = os.path.join(ROOT, "profiles", "k_row_stats_traffic.json")
+    """DRAM bytes (read + write) of one verify step of the bench workload from
+    the committed ncu capture (profiles/verify_step_traffic.json): per launch of
+    the sweep, and of the whole step (every kernel).  Valid only while the
+    kernel source is unchanged since the capture (checked by hash); None
+    otherwise."""
+    p = os.path.join(ROOT, "profiles", "verify_step_traffic.json")
     src = os.path.join(ROOT, "speculative_sampling_b200", "csrc", "specdec.cu")
     try:
         with open(p) as f:
@@ -86,14 +89,15 @@ def stored_traffic():
         h = hashlib.sha256(open(src, "rb").read()).hexdigest()
         if d.get("source_sha256") != h:
             return None
-        return d.get("traffic_bytes_per_launch")
+        return d
     except Exception:
         return None
 
 
 class ClockSampler:
-    """SM clock and throttle reasons of one GPU, sampled every 10 ms via NVML
-    while running."""
+    """SM clock and throttle reasons of one GPU, sampled via NVML while running:
+    every 10 ms, and back to back (no sleep) while ``fast`` is set, so that a
+    timed region of a millisecond still gets samples."""
 
     REASONS = {
         "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
@@ -117,7 +121,9 @@ class ClockSampler:
             self.nv = None
             self.err = str(e)
         self._stop = threading.Event()
+        self._wake = threading.Event()
         self._t = None
+        self.fast = False
 
     def _run(self):
         nv = self.nv
@@ -131,16 +137,29 @@ class ClockSampler:
                 self.samples.append((time.perf_counter(), mhz, r))
             except Exception as e:  # pragma: no cover
                 self.err = str(e)
-            self._stop.wait(0.01)
+            if not self.fast:
+                self._wake.wait(0.01)
+                self._wake.clear()
 
     def start(self):
         if self.nv is not None:
             self._t = threading.Thread(target=self._run, daemon=True)
             self._t.start()
 
+    def go_fast(self):
+        """Sample back to back from now on; returns once a fresh sample exists."""
+        self.fast = True
+        self._wake.set()
+        if self.nv is None or self._t is None:
+            return
+        t = time.perf_counter()
+        while (not self.samples or self.samples[-1][0] < t) and time.perf_counter() - t < 0.05:
+            time.sleep(0)
+
     def stop(self):
         if self._t is not None:
             self._stop.set()
+            self._wake.set()
             self._t.join()
 
     def summary(self):
@@ -303,6 +322,7 @@ def run_cuda(args):
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    sampler.go_fast()
     tw0 = time.perf_counter()
     e0.record(stream)
     for i in range(args.steps):
@@ -310,16 +330,39 @@ def run_cuda(args):
     e1.record(stream)
     torch.cuda.synchronize()
     tw1 = time.perf_counter()
+    sampler.fast = False
     barrier()
     sampler.window = (tw0, tw1)
     sampler.stop()
     after = [L.specdec_launch_count(i) for i in range(nk)]
     ms = sdist.max_over_ranks(e0.elapsed_time(e1), dev)
+    # step distribution: the same K steps again, each bracketed by its own pair
+    # of events on the stream (back to back, no synchronisation between steps)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for i in range(args.steps):
+        evs[i][0].record(stream)
+        step(i)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    per_step = np.array([a.elapsed_time(b) for a, b in evs]) * 1e3  # us
+    # single-call latency: one call at a time, synchronised before the next
+    lat = []
+    for i in range(min(args.steps, 100)):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step(i)
+        b.record(stream)
+        torch.cuda.synchronize()
+        lat.append(a.elapsed_time(b) * 1e3)
+    lat = np.array(lat)
     # kernel region: the same K steps again with every launch bracketed by CUDA
     # events on its stream; gives each kernel's mean device time (roofline)
     kern = {}
+    # launches of each kernel per step (the sweep runs once per wave of sequences)
+    lps = [(a - b) / args.steps for a, b in zip(after, before)]
     if args.kernel_timing == "on":
-        sd.profile_begin(args.steps)
+        sd.profile_begin(int(args.steps * max(lps)) + 1)
         for i in range(args.steps):
             step(i)
         torch.cuda.synchronize()
@@ -358,6 +401,46 @@ def run_cuda(args):
                  "tokens_equal_full_call": same_tokens,
                  "note": "value counts the full two-tensor floor per step, as the headline "
                          "does; read_GBs counts the rows this call actually reads"}
+        # the same shape at low acceptance (draft noise 1.5 for every sequence):
+        # the full call and early exit, each timed over the K steps
+        xl = sdist.generate_shard(args.workload, rank, world, sigma=1.5)
+        lb = [dict(t=tview(xl.target).to(dev), d=tview(xl.draft).to(dev),
+                   tok=torch.from_numpy(xl.tokens).to(dev),
+                   ua=torch.from_numpy(xl.u_accept).to(dev),
+                   ur=torch.from_numpy(xl.u_resample).to(dev),
+                   T=torch.from_numpy(xl.temperature).to(dev),
+                   ot=torch.empty((B, K + 1), dtype=torch.int32, device=dev),
+                   on=torch.empty((B,), dtype=torch.int32, device=dev)) for _ in range(ncopies)]
+        lcalls = [(b["t"].data_ptr(), b["d"].data_ptr(), b["tok"].data_ptr(), b["ua"].data_ptr(),
+                   b["ur"].data_ptr(), b["T"].data_ptr(), B, K, V, dt_code, b["ot"].data_ptr(),
+                   b["on"].data_ptr(), sp) for b in lb]
+        low = {}
+        for key, f in (("full_ms_per_step", fn), ("early_exit_ms_per_step", fe)):
+            for i in range(3):
+                if f(*lcalls[i % ncopies]) != 0:
+                    raise RuntimeError("verify failed on the low-acceptance batch")
+            torch.cuda.synchronize()
+            barrier()
+            torch.cuda.synchronize()
+            g0 = torch.cuda.Event(enable_timing=True)
+            g1 = torch.cuda.Event(enable_timing=True)
+            g0.record(stream)
+            for i in range(args.steps):
+                f(*lcalls[i % ncopies])
+            g1.record(stream)
+            torch.cuda.synchronize()
+            barrier()
+            low[key] = sdist.max_over_ranks(g0.elapsed_time(g1), dev) / args.steps
+            if key == "full_ms_per_step":
+                low_tok = lb[0]["ot"].cpu().numpy().copy()
+        n_l = lb[0]["on"].cpu().numpy()
+        rows_l = int(np.sum(np.where(n_l >= P, 2 * K + 1, 2 * P)))
+        low.update(rows_read_fraction=rows_l / (B * (2 * K + 1)),
+                   mean_accepted=float(np.mean(n_l)),
+                   tokens_equal_full_call=bool(np.array_equal(lb[0]["ot"].cpu().numpy(), low_tok)),
+                   note="the bench shape with draft noise 1.5 for every sequence")
+        early["low_acceptance"] = low
+        del lb, lcalls
 
     # ---- SMC-SD weight step on the same logits (groups of 8 particles) -------
     smc_line = None
@@ -525,16 +608,28 @@ def run_cuda(args):
         "gpu_launches": launches,
     }
     if kern:
+        # one verify step launches the sweep once per wave of sequences; the
+        # achieved rate is the algorithmic bytes of a launch over its mean time
         st_ms, st_n = kern["k_row_stats"]
+        per_launch = floor * args.steps / max(st_n, 1)
         avg = st_ms / max(st_n, 1)
-        ach = floor / (avg * 1e-3) / 1e9
+        ach = per_launch / (avg * 1e-3) / 1e9
+        tr = stored_traffic() if args.workload == "batched_b64_k5_v128256_bf16" else None
         line["roofline"] = {"bound": "hbm", "kernel": "k_row_stats", "achieved": ach,
                             "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                            "frac": ach / peak, "traffic": stored_traffic(),
-                            "algorithmic_bytes_per_launch": floor,
+                            "frac": ach / peak,
+                            "traffic": tr["sweep_bytes_per_launch"] if tr else None,
+                            "algorithmic_bytes_per_launch": per_launch,
+                            "launches_per_step": st_n / args.steps,
                             "launches_timed": st_n,
                             "timing": "CUDA events around each launch on its stream, over a "
                                       "second run of the K steps"}
+        if tr:
+            line["step_traffic"] = {"dram_bytes_per_step": tr["step_bytes"],
+                                    "algorithmic_bytes_per_step": floor,
+                                    "ratio": tr["step_bytes"] / floor,
+                                    "per_kernel": tr["per_kernel_bytes_per_step"],
+                                    "source": "profiles/verify_step_traffic.json"}
         line["kernel_us"] = {k: (v[0] / max(v[1], 1) * 1e3) for k, v in kern.items()}
     if early is not None:
         line["early_exit"] = early
@@ -546,7 +641,15 @@ def run_cuda(args):
         line["verify_chained"] = chained_line
     line["e2e"] = {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                    "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
+    line["step_us"] = {"median": float(np.median(per_step)), "p10": float(np.percentile(per_step, 10)),
+                       "p90": float(np.percentile(per_step, 90)), "steps": int(per_step.size),
+                       "note": "each of K back-to-back steps bracketed by its own events"}
+    line["latency_us"] = {"median": float(np.median(lat)), "p10": float(np.percentile(lat, 10)),
+                          "p90": float(np.percentile(lat, 90)), "calls": int(lat.size),
+                          "note": "one call at a time, the stream synchronised between calls"}
     line["clocks"] = sampler.summary()
+    if line["clocks"].get("sm_mhz"):
+        line["clocks"]["sm_mhz_x_us_per_step"] = line["clocks"]["sm_mhz"] * ms_step * 1e3
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(x, w, args.cpu_seconds)
     print(json.dumps(line), flush=True)

@@ -92,8 +92,9 @@ typedef enum specdec_dtype { SPECDEC_F32 = 0, SPECDEC_BF16 = 1 } specdec_dtype;
 #define SPECDEC_ERR_TOKEN 1u       /* a draft token outside [0, V)            */
 #define SPECDEC_ERR_TEMPERATURE 2u /* a temperature not finite and > 0        */
 #define SPECDEC_ERR_LOGITS 4u      /* a row with NaN / +Inf / only -Inf       */
-#define SPECDEC_ERR_TIMEOUT 8u     /* a bounded on-chip wait ran out: the
-                                      call's outputs are all -1              */
+#define SPECDEC_ERR_TIMEOUT 8u     /* a bounded on-chip wait ran out: every
+                                      sequence whose row statistics it left
+                                      incomplete gets outputs -1            */
 
 /* Optional diagnostics (device pointers, each nullable).  Row order per
  * sequence: target rows 0..K, then draft rows 0..K-1.
@@ -112,8 +113,9 @@ typedef struct specdec_debug {
 } specdec_debug;
 
 /* The verify step (see the top of this file).  Uses a workspace owned by the
- * library (one per device, grown on demand with cudaMalloc, which
- * synchronises the device the first time a size is seen). */
+ * library, one per (device, stream): calls on different streams may overlap on
+ * the GPU and never share one.  A workspace is grown on demand with cudaMalloc,
+ * which synchronises the device the first time a stream sees a larger size. */
 specdec_status specdec_verify(const void *target_logits, const void *draft_logits,
                               const int32_t *draft_tokens, const float *u_accept,
                               const float *u_resample, const float *temperature, int B, int K,
@@ -269,6 +271,22 @@ specdec_status specdec_verify_chained(
     int V, specdec_dtype dtype, int32_t *out_tokens, int32_t *out_num_emitted,
     int32_t *stage1_tokens, int32_t *stage1_num_accepted, void *stream);
 
+/* specdec_verify_chained with diagnostics of its second stage (dbg2 may be
+ * NULL; every field nullable, device memory):
+ *   row_max, row_sum [B, 2K+1]: entries 0..K are the final layer's rows
+ *     (max_v z_v and sum_v exp((z_v - max)/T)); entries K+1..2K are untouched;
+ *   p_x, q_x [B, K+1]: p_f,j(s_j) and q_i,j(s_j) for the positions j the
+ *     second stage tests (others untouched);
+ *   Z [B]: the mass sum_v max(0, p_f - q_i) of the second stage's draw
+ *     (untouched when all tested tokens are accepted). */
+specdec_status specdec_verify_chained_ex(
+    const void *final_logits, const void *intermediate_logits, const void *draft_logits,
+    const int32_t *draft_tokens, const float *u_accept1, const float *u_resample1,
+    const float *u_accept2, const float *u_resample2, const float *temperature, int B, int K,
+    int V, specdec_dtype dtype, int32_t *out_tokens, int32_t *out_num_emitted,
+    int32_t *stage1_tokens, int32_t *stage1_num_accepted, const specdec_debug *dbg2,
+    void *stream);
+
 /* End-to-end variant: every pointer is HOST memory (pinned memory makes the
  * copies asynchronous).  Copies the inputs to library-owned device buffers,
  * runs the verify step on `stream`, copies the outputs back and synchronises
@@ -282,6 +300,16 @@ specdec_status specdec_verify_host(const void *target_logits, const void *draft_
 /* Synchronise `stream`, then read and clear the current device's error word
  * (SPECDEC_ERR_* bits) into *flags.  Returns SPECDEC_EDEVICE when a bit was set. */
 specdec_status specdec_device_errors(void *stream, uint32_t *flags);
+
+/* The device error word as a status: synchronises the current device (all
+ * streams), reads and clears its error word, and returns SPECDEC_EDEVICE when
+ * any SPECDEC_ERR_* bit was set (specdec_device_errors gives the bits),
+ * SPECDEC_OK otherwise, SPECDEC_ECUDA when the synchronisation failed. */
+specdec_status specdec_get_error(void);
+
+/* A short English description of a status (a static string; never NULL).
+ * The same text as specdec_status_string. */
+const char *specdec_error_string(specdec_status s);
 
 /* Allocation-free verify (no counterpart on the pages: an interface addition).
  *
@@ -318,6 +346,27 @@ specdec_status specdec_verify_static(const void *target_logits, const void *draf
 void specdec_release(void);
 
 const char *specdec_status_string(specdec_status s);
+
+/* Testing hook of the failure path (no counterpart on the pages).  Every
+ * on-chip wait of the statistics sweep is bounded; when one runs out the
+ * kernel sets SPECDEC_ERR_TIMEOUT, marks the statistics it could not finish as
+ * incomplete and winds down, and the sequences depending on them get outputs
+ * -1, so the device stays usable.  This hook makes that path testable without
+ * a fault: wait_ns sets the bound of every wait in later launches (default
+ * 2e9 ns), and skip_tile >= 0 makes the sweep's producer never issue the copy
+ * of that tile (its index within one sweep launch), so the waits for it run
+ * out.  specdec_test_set_wait_fault(-1, 2000000000) restores the defaults.
+ * SPECDEC_EINVAL for skip_tile < -1 or wait_ns == 0.  Not thread-safe with
+ * respect to calls in flight on other host threads. */
+specdec_status specdec_test_set_wait_fault(long long skip_tile, unsigned long long wait_ns);
+
+/* Testing hook of the statistics sweep's FMA-pipe exponential (no
+ * counterpart on the pages): y[i] = 2^a[i] for n device floats, computed by
+ * the same device function the sweep uses for part of its exponentials
+ * (argument reduction to [-1/2, 1/2] and a degree-5 minimax polynomial; valid
+ * for a <= 64, arguments below -125 give about 2^-125).  Asynchronous on
+ * `stream`.  SPECDEC_EINVAL for n < 0 or null pointers with n > 0. */
+specdec_status specdec_test_exp2(const float *a, float *y, int n, void *stream);
 
 /* Kernel accounting, for benchmarks.  The library has specdec_kernel_count()
  * kernels; specdec_kernel_name(i) names kernel i.  specdec_launch_count(i)

@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(PKG, "libspecdec.so")
 SPECDEC_OK, SPECDEC_EINVAL, SPECDEC_ECUDA, SPECDEC_EDEVICE, SPECDEC_ESTATE, SPECDEC_ESIZE = range(6)
 SPECDEC_STATIC_SCRATCH_BYTES = 4 << 20
 SPECDEC_F32, SPECDEC_BF16 = 0, 1
-SPECDEC_ERR_TOKEN, SPECDEC_ERR_TEMPERATURE, SPECDEC_ERR_LOGITS = 1, 2, 4
+SPECDEC_ERR_TOKEN, SPECDEC_ERR_TEMPERATURE, SPECDEC_ERR_LOGITS, SPECDEC_ERR_TIMEOUT = 1, 2, 4, 8
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -41,7 +41,13 @@ _SIGS = {
     "specdec_topk_exclude": (_I, [_P, ctypes.c_longlong, _P, _I, _I, _I, _P, _I, _P, _P, _P]),
     "specdec_verify_chained": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P,
                                     _P, _P, _P]),
+    "specdec_verify_chained_ex": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P,
+                                       _P, _P, _P, _P, _P]),
     "specdec_device_errors": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
+    "specdec_get_error": (_I, []),
+    "specdec_error_string": (ctypes.c_char_p, [_I]),
+    "specdec_test_set_wait_fault": (_I, [ctypes.c_longlong, ctypes.c_ulonglong]),
+    "specdec_test_exp2": (_I, [_P, _P, _I, _P]),
     "specdec_release": (None, []),
     "specdec_status_string": (ctypes.c_char_p, [_I]),
     "specdec_kernel_count": (_I, []),
@@ -232,11 +238,23 @@ def specdec_verify_chained(final, inter, draft, tokens, u_accept1, u_resample1, 
                                         stage1_num_accepted, stream)
 
 
+def specdec_verify_chained_ex(final, inter, draft, tokens, u_accept1, u_resample1, u_accept2,
+                              u_resample2, temperature, B, K, V, dtype, out_tokens,
+                              out_num_emitted, stage1_tokens, stage1_num_accepted, dbg2,
+                              stream) -> int:
+    return lib().specdec_verify_chained_ex(final, inter, draft, tokens, u_accept1, u_resample1,
+                                           u_accept2, u_resample2, temperature, B, K, V, dtype,
+                                           out_tokens, out_num_emitted, stage1_tokens,
+                                           stage1_num_accepted, dbg2, stream)
+
+
 def verify_chained(final, inter, draft, tokens, u_accept1, u_resample1, u_accept2, u_resample2,
-                   temperature, stream=None) -> dict:
+                   temperature, stream=None, debug2: Optional[dict] = None) -> dict:
     """Chained two-stage verify on CUDA tensors (see specdec_verify_chained).
     Returns a dict of CUDA int32 tensors: out_tokens [B,K+1], num_emitted [B],
-    stage1_tokens [B,K+1], stage1_n [B]."""
+    stage1_tokens [B,K+1], stage1_n [B].  With ``debug2`` (a dict of
+    preallocated tensors named as specdec_debug's fields) the call goes through
+    specdec_verify_chained_ex and fills the second stage's diagnostics."""
     import torch
     B, K1, V = final.shape
     K = K1 - 1
@@ -249,14 +267,21 @@ def verify_chained(final, inter, draft, tokens, u_accept1, u_resample1, u_accept
                temperature)
     if stream is None:
         stream = torch.cuda.current_stream(dev).cuda_stream
-    st = specdec_verify_chained(final.data_ptr(), inter.data_ptr(), draft.data_ptr(),
-                                tokens.data_ptr(), u_accept1.data_ptr(), u_resample1.data_ptr(),
-                                u_accept2.data_ptr(), u_resample2.data_ptr(),
-                                temperature.data_ptr(), B, K, V, _dtype_code(final),
-                                out["out_tokens"].data_ptr(), out["num_emitted"].data_ptr(),
-                                out["stage1_tokens"].data_ptr(), out["stage1_n"].data_ptr(),
-                                stream)
-    _chk(st, "specdec_verify_chained")
+    dbg = None
+    if debug2 is not None:
+        d = _Debug()
+        for f, _ in _Debug._fields_:
+            t = debug2.get(f)
+            setattr(d, f, t.data_ptr() if t is not None else None)
+        dbg = ctypes.byref(d)
+    st = specdec_verify_chained_ex(final.data_ptr(), inter.data_ptr(), draft.data_ptr(),
+                                   tokens.data_ptr(), u_accept1.data_ptr(), u_resample1.data_ptr(),
+                                   u_accept2.data_ptr(), u_resample2.data_ptr(),
+                                   temperature.data_ptr(), B, K, V, _dtype_code(final),
+                                   out["out_tokens"].data_ptr(), out["num_emitted"].data_ptr(),
+                                   out["stage1_tokens"].data_ptr(), out["stage1_n"].data_ptr(),
+                                   dbg, stream)
+    _chk(st, "specdec_verify_chained_ex")
     return out
 
 
@@ -264,6 +289,22 @@ def specdec_device_errors(stream=None) -> tuple:
     flags = ctypes.c_uint32(0)
     st = lib().specdec_device_errors(stream, ctypes.byref(flags))
     return st, int(flags.value)
+
+
+def specdec_get_error() -> int:
+    return lib().specdec_get_error()
+
+
+def specdec_error_string(status: int) -> str:
+    return lib().specdec_error_string(int(status)).decode()
+
+
+def specdec_test_set_wait_fault(skip_tile: int, wait_ns: int) -> int:
+    return lib().specdec_test_set_wait_fault(int(skip_tile), int(wait_ns))
+
+
+def specdec_test_exp2(a, y, n, stream) -> int:
+    return lib().specdec_test_exp2(a, y, n, stream)
 
 
 def specdec_release() -> None:

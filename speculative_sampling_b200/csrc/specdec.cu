@@ -11,8 +11,8 @@
 //                   into a 3-stage shared-memory ring (full/empty mbarriers,
 //                   every wait bounded); 8 consumer warps fold them into
 //                   split-V softmax statistics (row max m, sum of 2^((z-m)*c))
-//                   and write one partial per warp and row segment.  It streams
-//                   the whole input once and is the HBM-bound kernel.
+//                   and each CTA writes one partial per row segment.  It
+//                   streams the whole input once and is the HBM-bound kernel.
 //   k_finish        per sequence, on several CTAs: combines the partials of the
 //                   2K+1 rows in fp64, gathers p_i(x_i), q_i(x_i), tests
 //                   u*q < p on K lanes (__ballot_sync/__ffs), writes the
@@ -23,9 +23,10 @@
 //   k_smc_resample  SMC-SD: log-weights, effective sample size and systematic
 //                   resampling per group of particles.
 //   k_topk_exclude  top-k token ids of a row leaving one token out.
-// The verify kernels are launched with programmatic dependent launch: each
-// signals its dependents at its start and waits for its predecessor
-// (cudaGridDependencySynchronize) only where it first needs its results.
+// Kernels are launched with programmatic dependent launch: each signals its
+// dependents at its start and waits for its predecessor
+// (cudaGridDependencySynchronize) only where it first needs its results; the
+// call's first kernel waits before it reads anything.
 //
 // Arithmetic: logits are widened exactly to fp32.  Exponentials are
 // 2^((z - m) * c) with c = log2(e)/T carried as an fp32 pair (hi + lo, with
@@ -44,7 +45,9 @@
 
 #include <cfloat>
 #include <climits>
+#include <atomic>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <string>
 #include <unordered_map>
@@ -170,23 +173,24 @@ __device__ __forceinline__ float warp_max_nan(float v) {
 // ---------------------------------------------------------------------------
 // kernel 1: softmax statistics of every row
 // ---------------------------------------------------------------------------
-// The B*(2K+1) rows are cut into units: a unit is UT consecutive tiles of one
-// row; a tile is CW*32*U 16-byte vectors (16 KB for U = 4).  CTA g of a grid
-// of G handles units g, g+G, g+2G, ... so the grid sweeps the logits front to
-// back, sequence after sequence.
+// A sweep reads the rows of a range of sequences (a wave of the batch), in
+// sequence order, cut into tiles of CW*32*U 16-byte vectors (16 KB for U = 4);
+// CTA g of a grid of G owns the contiguous tile range [g*T/G, (g+1)*T/G).
 //
 // Warp specialisation: one producer warp streams tiles with cp.async.bulk
-// (the TMA bulk-copy engine; plain CTA-local copies, no multicast) into an
-// NSTAGE-deep ring in shared memory, tracked by "full" / "empty" mbarriers;
-// CW consumer warps take a tile out of the ring (one 16-byte shared load per
-// vector), release the slot, and fold it into a per-thread (max, sum) in
-// registers.  A unit's setup (row pointer, alignment, log2(e)/T) and its
-// CTA combine are paid once per unit.  Per element the consumers spend one
-// exact bf16->fp32 unpack, one FMNMX for the tile max, three packed fp32x2
-// operations at half an issue slot each, one MUFU ex2 and half a packed add.
-// Every wait is bounded: a wait that runs out sets SPECDEC_ERR_TIMEOUT in the
-// device error word and the kernel winds down (the producer first waits, again
-// bounded, for the copies it has in flight).
+// (the TMA bulk-copy engine; each CTA copies only into its own shared memory)
+// into an NSTAGE-deep ring in shared memory, tracked by "full" / "empty"
+// mbarriers; CW consumer warps take a tile out of the ring (one 16-byte shared
+// load per vector), release the slot, and fold it into a per-thread (max, sum)
+// in registers.  At the end of each row segment (the CTA's tiles of one row)
+// the warps' statistics are combined into one partial per CTA.  Per element
+// the consumers spend one exact bf16->fp32 unpack, one FMNMX for the tile max,
+// three packed fp32x2 operations at half an issue slot each, one exponential
+// (MUFU ex2, or for SPECDEC_EXP_FMA_PAIRS pairs per vector the FMA-pipe
+// polynomial) and half a packed add.  Every wait is bounded: a wait that runs
+// out sets SPECDEC_ERR_TIMEOUT in the device error word, the CTA's partials
+// from then on are marked incomplete, and the kernel winds down (the producer
+// first waits, again bounded, for the copies it has in flight).
 
 #ifndef SPECDEC_SWEEP_WARPS
 #define SPECDEC_SWEEP_WARPS 8
@@ -194,15 +198,28 @@ __device__ __forceinline__ float warp_max_nan(float v) {
 #ifndef SPECDEC_SWEEP_CTAS_PER_SM
 #define SPECDEC_SWEEP_CTAS_PER_SM 3
 #endif
+// Registers per thread of the sweep (0: the compiler's choice under the
+// launch bound of kStatsCtasPerSm CTAs per SM).
+#ifndef SPECDEC_SWEEP_MAXNREG
+#define SPECDEC_SWEEP_MAXNREG 0
+#endif
 constexpr int CW = SPECDEC_SWEEP_WARPS;  // consumer warps of a sweep CTA
 constexpr int NTC = CW * 32;        // consumer threads
 constexpr int NTS = NTC + 32;       // + one producer warp
 constexpr int NSTAGE = 3;           // depth of the shared-memory ring
-constexpr unsigned long long kWaitNs = 2000000000ull;  // a wait gives up after 2 s
+constexpr unsigned long long kWaitNs = 2000000000ull;  // a wait gives up after 2 s by default
 constexpr unsigned kSuspendNs = 20000;  // longest sleep of one try_wait round
 constexpr int kStatsCtasPerSm = SPECDEC_SWEEP_CTAS_PER_SM;  // sweep CTAs per SM the grid is sized for
 constexpr int kFinishUW = 4;        // vectors per lane in a k_finish chunk
-constexpr int kFinishCtasPerSm = 4; // k_finish grids fit one wave of this many CTAs per SM
+constexpr int kFinishThreads = 256;   // threads of a k_finish CTA
+constexpr int kFinishCtasPerSm = 4;   // k_finish grids fit one wave of this many CTAs per SM
+constexpr int kFinishMaxNreg = 64;    // k_finish registers per thread (launch bound below)
+// A sweep combines its warps' partials per CTA when a row can meet more than
+// this many of its CTAs.
+#ifndef SPECDEC_CTA_COMBINE_SLOTS
+#define SPECDEC_CTA_COMBINE_SLOTS 4
+#endif
+constexpr int kCtaCombineSlots = SPECDEC_CTA_COMBINE_SLOTS;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -237,16 +254,23 @@ __device__ __forceinline__ unsigned long long global_ns() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
-// bounded wait for the phase of the given parity; false when it ran out (the
-// bound is wall-clock time, so it does not depend on how long a round sleeps)
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, unsigned parity) {
+// bounded wait for the phase of the given parity; false when it ran out after
+// limit_ns (the bound is wall-clock time, so it does not depend on how long a
+// round sleeps)
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, unsigned parity,
+                                          unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   do {
     if (mbar_try_wait(bar, parity)) return true;
-  } while (global_ns() - t0 < kWaitNs);
+  } while (global_ns() - t0 < limit_ns);
   atomicOr(&g_error_flags, SPECDEC_ERR_TIMEOUT);
   return false;
+}
+// barrier of the consumer warps of a sweep CTA only (the producer warp is not
+// part of it)
+__device__ __forceinline__ void consumer_sync() {
+  asm volatile("bar.sync 1, %0;" ::"r"(NTC) : "memory");
 }
 // global -> shared bulk copy completing on an mbarrier (16-byte aligned
 // addresses, size a multiple of 16)
@@ -276,6 +300,44 @@ struct Pairs<float> {
                   : make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
   }
 };
+
+// 2^a for a pair of arguments on the FMA pipe instead of the MUFU unit: the
+// sweep evaluates part of its exponentials this way so that the two pipes
+// share the work.  Method (the standard software exponential): split
+// a = n + f with n = round(a) (adding 1.5 * 2^23 rounds to an integer in the
+// low mantissa bits; n and f = a - n are exact) and f in [-1/2, 1/2]; 2^f by a
+// degree-5 polynomial whose coefficients minimise the maximum relative error
+// on [-1/2, 1/2] (Remez exchange, fitted in fp64 and rounded to fp32: 7.5e-8
+// relative error in exact arithmetic, 2.2e-7 = 3.6 ulp including the fp32
+// Horner steps, against 2 ulp for ex2.approx); then 2^n is applied by adding
+// n to the exponent field.  Arguments below -125 are clamped there (so every
+// result is a normal number): such a term, about 2^-125 instead of less, is far
+// below the resolution of the sums it enters, which are at least 1.  Valid for
+// a <= 64.
+constexpr float kExp2C0 = 1.0000001192092896f, kExp2C1 = 0.6931469440460205f,
+                kExp2C2 = 0.24022120237350464f, kExp2C3 = 0.05550713092088699f,
+                kExp2C4 = 0.009675540961325169f, kExp2C5 = 0.0013276472454890609f;
+__device__ __forceinline__ float2 exp2_fma2(float2 a) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  a.x = fmaxf(a.x, -125.0f);
+  a.y = fmaxf(a.y, -125.0f);
+  const float2 t = __fadd2_rn(a, make_float2(kRound, kRound));
+  const float2 n = __fadd2_rn(t, make_float2(-kRound, -kRound));
+  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), a);
+  float2 p = __ffma2_rn(make_float2(kExp2C5, kExp2C5), f, make_float2(kExp2C4, kExp2C4));
+  p = __ffma2_rn(p, f, make_float2(kExp2C3, kExp2C3));
+  p = __ffma2_rn(p, f, make_float2(kExp2C2, kExp2C2));
+  p = __ffma2_rn(p, f, make_float2(kExp2C1, kExp2C1));
+  p = __ffma2_rn(p, f, make_float2(kExp2C0, kExp2C0));
+  // (bits of t) << 23 is n << 23: the rounding constant's own bits shift out
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+// pairs of each 16-byte vector whose exponentials the sweep takes on the FMA
+// pipe (the rest on MUFU)
+#ifndef SPECDEC_EXP_FMA_PAIRS
+#define SPECDEC_EXP_FMA_PAIRS 0
+#endif
 
 __device__ __forceinline__ float fmax3_nan(float a, float b, float c) {
   float y;
@@ -349,7 +411,10 @@ __device__ __forceinline__ void vec_fold(const uint4 &v, RunStat &q, Scale c, fl
   for (int k = 0; k < N; ++k) {
     const float2 d = __fadd2_rn(x[k], nr);
     const float2 a = __ffma2_rn(d, hi, __fmul2_rn(d, lo));
-    e[k] = make_float2(ex2(a.x), ex2(a.y));
+    if (k < SPECDEC_EXP_FMA_PAIRS)
+      e[k] = exp2_fma2(a);
+    else
+      e[k] = make_float2(ex2(a.x), ex2(a.y));
   }
 #pragma unroll
   for (int w = 1; w < N; w *= 2)
@@ -382,6 +447,13 @@ struct StatsGeom {
   int d_rows;       // rows per sequence of the draft tensor (K, or K+1 when it is an
                     // intermediate verifier's logits)
   int tonly;        // the window holds target rows p0 .. p0+np-1 only (rps = np)
+  unsigned long long wait_ns;  // bound of every on-chip wait
+  long long skip_tile;         // test hook: the producer never issues this tile's copy
+                               // (-1: none), so a consumer wait runs out
+  int nb;           // sequences of this sweep
+  int pcw;          // partials per (row, CTA): CW (one per consumer warp, no CTA
+                    // barrier) or 1 (the warps' partials combined per CTA, for rows
+                    // shared by many CTAs, so that the finish pass reads fewer)
 };
 __device__ __forceinline__ bool seq_active(const StatsGeom &g, long long b) {
   return g.state == nullptr || __ldcg(g.state + b) == kSeqActive;
@@ -395,7 +467,10 @@ __host__ __device__ __forceinline__ long long tile_begin(long long g, long long 
   return g * T / G;
 }
 __host__ __device__ __forceinline__ long long tile_owner(long long t, long long G, long long T) {
-  return ((t + 1) * G - 1) / T;
+  const long long num = (t + 1) * G - 1;
+  // (a 32-bit division where the operands fit: far cheaper than a 64-bit one)
+  if (num < 4294967296LL && T < 4294967296LL) return (long long)((unsigned)num / (unsigned)T);
+  return num / T;
 }
 
 // The current row of a CTA's tile walk.  Rows are numbered b*rps + w, w the
@@ -435,18 +510,35 @@ struct RowCursor {
   }
 };
 
+#if SPECDEC_SWEEP_MAXNREG > 0
+#define SPECDEC_SWEEP_BOUNDS __maxnreg__(SPECDEC_SWEEP_MAXNREG)
+#else
+#define SPECDEC_SWEEP_BOUNDS __launch_bounds__(NTS, kStatsCtasPerSm)
+#endif
+
+// The partials of one row segment: one per consumer warp (pcw = CW), or the
+// CW warps' (max, sum) pairs combined in warp order with fp64 rescales (pcw =
+// 1); pad = 1 marks a partial left incomplete because a wait of this CTA ran
+// out.
+// Programmatic dependent launch: the grid may be placed while the kernel
+// before it on the stream drains; every thread waits for that kernel
+// (cudaGridDependencySynchronize) after the shared-memory setup, before it
+// reads an input or touches the workspace, and only then lets the dependent
+// finish pass launch.
 template <typename T, int U>
-__global__ void __launch_bounds__(NTS, kStatsCtasPerSm) k_row_stats(const T *__restrict__ target,
-                                                   const T *__restrict__ draft,
-                                                   const float *__restrict__ temperature,
-                                                   StatsGeom g, Partial *__restrict__ part,
-                                                   unsigned *__restrict__ tickets, int B) {
+__global__ void SPECDEC_SWEEP_BOUNDS k_row_stats(const T *__restrict__ target,
+                                                 const T *__restrict__ draft,
+                                                 const float *__restrict__ temperature,
+                                                 StatsGeom g, Partial *__restrict__ part,
+                                                 unsigned *__restrict__ tickets, int B) {
   constexpr int VEC = Dt<T>::VEC;
   constexpr long long TV = (long long)NTC * U;  // vectors per tile
   constexpr unsigned TILE_BYTES = (unsigned)TV * 16u;
   extern __shared__ __align__(128) unsigned char ring[];  // NSTAGE * TILE_BYTES
   __shared__ __align__(8) uint64_t full[NSTAGE], empty[NSTAGE];
   __shared__ int s_abort;
+  __shared__ float s_wm[2][CW];   // per-warp partials of the last two row segments
+  __shared__ double s_ws[2][CW];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long G = gridDim.x;
   const long long t0 = tile_begin(blockIdx.x, G, g.tiles);
@@ -461,19 +553,13 @@ __global__ void __launch_bounds__(NTS, kStatsCtasPerSm) k_row_stats(const T *__r
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  // This grid is launched with programmatic dependent launch: up to here it may
-  // overlap the kernel before it on the stream (the previous call's k_finish,
-  // which reads this workspace, or whatever wrote the inputs).  From here on
-  // every such kernel has completed and its writes are visible.
   cudaGridDependencySynchronize();
-  // the arrival tickets of k_finish (which runs after this kernel) start at 0
-  if (blockIdx.x == 0)
-    for (int i = threadIdx.x; i < B; i += blockDim.x) tickets[i] = 0u;
-  // Let the dependent k_finish grid launch now: its CTAs take the SM slots this
-  // grid's CTAs free as they finish and do their input gathers during the
-  // sweep's tail.  They read this kernel's results only after
-  // cudaGridDependencySynchronize, which waits for the whole grid to complete.
+  // the dependent finish pass may be placed now; it reads this kernel's
+  // results only after its own cudaGridDependencySynchronize
   cudaTriggerProgrammaticLaunchCompletion();
+  // the arrival tickets of the finish pass start at 0
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < g.nb; i += blockDim.x) tickets[i] = 0u;
   if (t0 >= t1) return;
 
   // The CTA's tiles [t0, t1) are walked as row segments: the tiles of one row
@@ -483,8 +569,10 @@ __global__ void __launch_bounds__(NTS, kStatsCtasPerSm) k_row_stats(const T *__r
 
   if (warp == CW) {  // ---------------- producer warp ----------------
     if (lane != 0) return;
-    unsigned it = 0, ph = 0;  // copies issued; phase parity of the current ring pass
-    int st = 0;               // ring slot of the next copy
+    unsigned ph = 0;  // phase parity of the current ring pass
+    int st = 0;       // ring slot of the next copy
+    // per slot: whether a copy was issued into it and the parity of its phase
+    unsigned pend = 0, pend_ph = 0;
     RowCursor<T> rc;
     rc.start(target, draft, g, t0);
     for (long long row = row_first; row <= row_last; ++row) {
@@ -496,14 +584,17 @@ __global__ void __launch_bounds__(NTS, kStatsCtasPerSm) k_row_stats(const T *__r
         const long long v0 = (long long)ti * TV;
         const long long v1 = (v0 + TV < rc.nvec) ? v0 + TV : rc.nvec;
         if (v0 >= v1) break;  // the rest of the row is its scalar tail
-        if (*(volatile int *)&s_abort || !mbar_wait(&empty[st], ph ^ 1u)) {
+        if (*(volatile int *)&s_abort || !mbar_wait(&empty[st], ph ^ 1u, g.wait_ns)) {
           atomicExch(&s_abort, 1);
           goto drain;
         }
-        const unsigned bytes = (unsigned)(v1 - v0) * 16u;
-        mbar_arrive_tx(&full[st], bytes);
-        bulk_load(ring + (size_t)st * TILE_BYTES, rc.pv + v0, bytes, &full[st]);
-        ++it;
+        if (row * g.tpr + ti != g.skip_tile) {
+          const unsigned bytes = (unsigned)(v1 - v0) * 16u;
+          mbar_arrive_tx(&full[st], bytes);
+          bulk_load(ring + (size_t)st * TILE_BYTES, rc.pv + v0, bytes, &full[st]);
+          pend |= 1u << st;
+          pend_ph = (pend_ph & ~(1u << st)) | (ph << st);
+        }
         if (++st == NSTAGE) {
           st = 0;
           ph ^= 1u;
@@ -513,23 +604,24 @@ __global__ void __launch_bounds__(NTS, kStatsCtasPerSm) k_row_stats(const T *__r
   drain:
     // The CTA must not retire with copies in flight: wait (bounded) until the
     // last copy issued into each slot has landed.
-    for (unsigned k = 0; k < NSTAGE && k < it; ++k) {
-      const unsigned j = it - 1 - k;
-      mbar_wait(&full[j % NSTAGE], (j / NSTAGE) & 1u);
-    }
+    for (int k = 0; k < NSTAGE; ++k)
+      if (pend & (1u << k)) mbar_wait(&full[k], (pend_ph >> k) & 1u, g.wait_ns);
     return;
   }
 
   // ---------------- consumer warps ----------------
-  // No CTA-wide barrier inside the walk: each warp folds its share of every
-  // tile and, at the end of a row segment, reduces its lanes and writes its own
-  // partial.  After an abort the waits and the arithmetic are skipped (every
-  // warp still walks the same tiles).
+  // Each warp folds its share of every tile.  At the end of a row segment the
+  // warps' partials are combined through shared memory (consumer-only barrier)
+  // and warp 0 writes one partial for the CTA.  After an abort the waits and
+  // the arithmetic are skipped (every warp still walks the same tiles) and the
+  // CTA's partials are marked incomplete.
   unsigned ph = 0;  // phase parity of the current ring pass
   int st = 0;       // ring slot of the next tile
+  int seg = 0;      // row segments finished (selects the s_wm / s_ws buffer)
   RowCursor<T> rc;
   rc.start(target, draft, g, t0);
-  Scale c = make_scale(kLog2e / (double)__ldg(temperature + rc.b));
+  float Tcur = __ldg(temperature + rc.b);
+  Scale c = make_scale(kLog2e / (double)Tcur);
   float thr = 64.0f / c.hi;
   // temperature of the sequence after this one, fetched a row ahead
   float T_next = (rc.b + 1 < B) ? __ldg(temperature + rc.b + 1) : 1.0f;
@@ -538,7 +630,8 @@ __global__ void __launch_bounds__(NTS, kStatsCtasPerSm) k_row_stats(const T *__r
       const bool new_seq = (rc.w == g.rps - 1);
       rc.next_row(target, draft, g);
       if (new_seq) {
-        c = make_scale(kLog2e / (double)T_next);
+        Tcur = T_next;
+        c = make_scale(kLog2e / (double)Tcur);
         thr = 64.0f / c.hi;
         T_next = (rc.b + 1 < B) ? __ldg(temperature + rc.b + 1) : 1.0f;
       }
@@ -554,7 +647,7 @@ __global__ void __launch_bounds__(NTS, kStatsCtasPerSm) k_row_stats(const T *__r
     for (int ti = tb; ti < tf; ++ti) {
       bool have = false;
       if (!*(volatile int *)&s_abort) {
-        have = __all_sync(FULL, mbar_wait(&full[st], ph));
+        have = __all_sync(FULL, mbar_wait(&full[st], ph, g.wait_ns));
         if (!have && lane == 0) atomicExch(&s_abort, 1);
       }
       const uint4 *tile = reinterpret_cast<const uint4 *>(ring + (size_t)st * TILE_BYTES);
@@ -577,7 +670,7 @@ __global__ void __launch_bounds__(NTS, kStatsCtasPerSm) k_row_stats(const T *__r
       const long long nv = rc.nvec - (long long)tpb * TV;
       bool have = false;
       if (!*(volatile int *)&s_abort) {
-        have = __all_sync(FULL, mbar_wait(&full[st], ph));
+        have = __all_sync(FULL, mbar_wait(&full[st], ph, g.wait_ns));
         if (!have && lane == 0) atomicExch(&s_abort, 1);
       }
       const uint4 *tile = reinterpret_cast<const uint4 *>(ring + (size_t)st * TILE_BYTES);
@@ -612,13 +705,47 @@ __global__ void __launch_bounds__(NTS, kStatsCtasPerSm) k_row_stats(const T *__r
     const float mw = warp_max_nan(m);
     double sw = (m == -INFINITY) ? 0.0 : (double)sl * (double)ex2(scaled(m - mw, c));
     sw = warp_sum(sw);
+    if (g.pcw != 1) {
+      // one partial per warp: no CTA barrier (a warp that skipped a tile has
+      // seen the abort flag by now)
+      if (lane == 0) {
+        const int aborted = *(volatile int *)&s_abort;
+        const long long slot = (long long)blockIdx.x - tile_owner(row * g.tpr, G, g.tiles);
+        Partial out;
+        out.s = aborted ? 0.0 : sw;
+        out.m = aborted ? __int_as_float(0x7fc00000) : mw;
+        out.pad = aborted ? 1u : 0u;
+        part[(row * g.slots + slot) * CW + warp] = out;
+      }
+      continue;
+    }
+    const int pb = seg & 1;
     if (lane == 0) {
-      const long long slot = (long long)blockIdx.x - tile_owner(row * g.tpr, G, g.tiles);
-      Partial out;
-      out.s = sw;
-      out.m = mw;
-      out.pad = 0;
-      part[(row * g.slots + slot) * CW + warp] = out;
+      s_wm[pb][warp] = mw;
+      s_ws[pb][warp] = sw;
+    }
+    // (two buffers: a warp writing the next segment's values has passed this
+    // barrier again only after warp 0 has read these)
+    consumer_sync();
+    ++seg;
+    if (warp == 0) {
+      // the CTA's partial: the warps' sums rescaled to their common max in
+      // fp64, added in warp order
+      const float mi = lane < CW ? s_wm[pb][lane] : -INFINITY;
+      const double si = lane < CW ? s_ws[pb][lane] : 0.0;
+      const float M = warp_max_nan(mi);
+      const double c64 = kLog2e / (double)Tcur;
+      double t = (mi == -INFINITY) ? si : si * exp2(((double)mi - (double)M) * c64);
+      t = warp_sum(t);
+      const int aborted = *(volatile int *)&s_abort;
+      if (lane == 0) {
+        const long long slot = (long long)blockIdx.x - tile_owner(row * g.tpr, G, g.tiles);
+        Partial out;
+        out.s = aborted ? 0.0 : t;
+        out.m = aborted ? __int_as_float(0x7fc00000) : M;
+        out.pad = aborted ? 1u : 0u;
+        part[(row * g.slots + slot) * CW] = out;
+      }
     }
   }
 }
@@ -649,19 +776,53 @@ struct DrawRow {
 // r = St * max(0, p - q) = max(0, e_t - (St/Sd) e_d) with e = 2^((z - m)c)
 // (or e_t for the bonus row).  The same inlined arithmetic serves the chunk
 // sums and the rescan, so both see bit-identical per-element weights.
+#ifndef SPECDEC_FINISH_EXP_FMA
+#define SPECDEC_FINISH_EXP_FMA 0
+#endif
+#ifndef SPECDEC_COMBINE_FP32
+#define SPECDEC_COMBINE_FP32 0
+#endif
 __device__ __forceinline__ float res_weight(float zt, float zd, const DrawRow &d) {
   const float et = ex2(scaled(zt - d.Mt, d.c));
   if (d.bonus) return et;
+#if SPECDEC_FINISH_EXP_FMA
+  // the draft row's exponential on the FMA pipe (the MUFU unit takes the
+  // target's): the finish pass is MUFU-bound
+  const float ed = exp2_fma2(make_float2(scaled(zd - d.Md, d.c), -125.0f)).x;
+#else
   const float ed = ex2(scaled(zd - d.Md, d.c));
+#endif
   const float t1 = __fmaf_rn(-d.lhi, ed, et);
   const float t2 = __fmaf_rn(-d.llo, ed, t1);
   return t2 > 0.0f ? t2 : 0.0f;
 }
+// The same weights for two adjacent entries with packed fp32x2 operations:
+// each lane of every packed operation rounds exactly as the scalar one above
+// (a - b is a + (-b) exactly), so the weights are bit-identical.
+__device__ __forceinline__ float2 res_weight2(float2 zt, float2 zd, const DrawRow &d) {
+  const float2 hi = make_float2(d.c.hi, d.c.hi), lo = make_float2(d.c.lo, d.c.lo);
+  const float2 dt = __fadd2_rn(zt, make_float2(-d.Mt, -d.Mt));
+  const float2 at = __ffma2_rn(dt, hi, __fmul2_rn(dt, lo));
+  const float2 et = make_float2(ex2(at.x), ex2(at.y));
+  if (d.bonus) return et;
+  const float2 dd = __fadd2_rn(zd, make_float2(-d.Md, -d.Md));
+  const float2 ad = __ffma2_rn(dd, hi, __fmul2_rn(dd, lo));
+#if SPECDEC_FINISH_EXP_FMA
+  const float2 ed = exp2_fma2(ad);
+#else
+  const float2 ed = make_float2(ex2(ad.x), ex2(ad.y));
+#endif
+  const float2 t1 = __ffma2_rn(make_float2(-d.lhi, -d.lhi), ed, et);
+  const float2 t2 = __ffma2_rn(make_float2(-d.llo, -d.llo), ed, t1);
+  return make_float2(t2.x > 0.0f ? t2.x : 0.0f, t2.y > 0.0f ? t2.y : 0.0f);
+}
 
 // Block-wide exclusive prefix sum of one double per thread, in thread order
-// (fixed association); `total` receives the block sum.  All threads call it.
+// (fixed association); `total` receives the block sum.  All NTH threads call it.
+template <int NTH>
 __device__ __forceinline__ double block_excl_scan(double v, double &total) {
-  __shared__ double sm[NWARP];
+  constexpr int NW = NTH / 32;
+  __shared__ double sm[NW];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   double incl = v;
 #pragma unroll
@@ -675,7 +836,7 @@ __device__ __forceinline__ double block_excl_scan(double v, double &total) {
   if (lane == 31) sm[warp] = incl;
   __syncthreads();
   double base = 0.0, tot = 0.0;
-  for (int w = 0; w < NWARP; ++w) {
+  for (int w = 0; w < NW; ++w) {
     if (w < warp) base += sm[w];
     tot += sm[w];
   }
@@ -693,11 +854,11 @@ __device__ __forceinline__ double prob64(const T *row, long long v, float M, dou
 // (contiguous segments per thread, block scan, first crossing).  If the fp64
 // residual is zero as well, draws from p (as the oracle does).  Used only when
 // the fp32 residual weights have run out of range.
-template <typename T>
+template <typename T, int NTH>
 __device__ __noinline__ int draw_exact64(const T *pt, const T *pd, long long V, float Mt,
                                          double St, float Md, double Sd, double c64, double u,
                                          int *s_y, int *s_lastpos, double *dbg_Z) {
-  const long long E = (V + NT - 1) / NT;
+  const long long E = (V + NTH - 1) / NTH;
   const long long e0 = (long long)threadIdx.x * E < V ? (long long)threadIdx.x * E : V;
   const long long e1 = (e0 + E < V) ? e0 + E : V;
   double sr = 0.0, sp = 0.0;
@@ -708,8 +869,8 @@ __device__ __noinline__ int draw_exact64(const T *pt, const T *pd, long long V, 
     sp += p;
   }
   double Zr, Zp;
-  const double xr = block_excl_scan(sr, Zr);
-  const double xp = block_excl_scan(sp, Zp);
+  const double xr = block_excl_scan<NTH>(sr, Zr);
+  const double xp = block_excl_scan<NTH>(sp, Zp);
   const bool use_p = !(Zr > 0.0);
   const double Z = use_p ? Zp : Zr;
   const double t = u * Z;
@@ -762,6 +923,8 @@ struct FinishWindow {
   double *dlogw;
   const int32_t *len;
   int emit_count;
+  int dbg_pstride;  // positions per sequence of the p_x / q_x diagnostics (K, or K+1
+                    // for a chained second stage)
   // Row statistics kept across passes (the chained verify): with `save_t` set,
   // the combined (max, sum) of every target row of the window is stored at
   // save_t[b*(K+1) + position]; with `dstat` set, the sweep covered only the
@@ -773,12 +936,12 @@ struct FinishWindow {
 };
 constexpr int kChainAll = -3;  // chained stage: every tested token accepted
 
-template <typename T, int UW>
-__global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
+template <typename T, int UW, int NTH>
+__global__ void __launch_bounds__(NTH, 65536 / (NTH * kFinishMaxNreg)) k_finish(
     const T *__restrict__ target, const T *__restrict__ draft,
     const int32_t *__restrict__ tokens, const float *__restrict__ u_accept,
     const float *__restrict__ u_resample, const float *__restrict__ temperature, int K,
-    long long V, int tpr, long long tiles, long long G1, int slots, int nsr, int cpb,
+    long long V, int tpr, long long tiles, long long G1, int slots, int pcw, int nsr, int cpb,
     int d_rows, int tok_stride, FinishWindow fw, const Partial *__restrict__ part,
     ResPartial *__restrict__ rpart, unsigned *__restrict__ counters,
     int32_t *__restrict__ out_tokens, int32_t *__restrict__ out_n,
@@ -787,10 +950,12 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
   constexpr int VEC = Dt<T>::VEC;
   constexpr long long CHV = 32LL * UW;                 // vectors per (warp-)chunk
   constexpr long long CH = CHV * VEC;                  // elements per chunk
-  constexpr int EMAX = (int)((CH + 2 * VEC + NT - 1) / NT);  // rescan elements per thread
+  constexpr int NW = NTH / 32;
+  constexpr int EMAX = (int)((CH + 2 * VEC + NTH - 1) / NTH);  // rescan elements per thread
   __shared__ float sM[66];
   __shared__ double sS[66];
   __shared__ int s_n, s_last, s_mode, s_chunk, s_y, s_lastpos;
+  __shared__ unsigned s_tmo[NW];  // per warp: a partial it read was marked incomplete
   __shared__ double s_base, s_t;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int ncb = (nsr + cpb - 1) / cpb;  // CTAs per sequence
@@ -802,6 +967,10 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
   // or the SMC-SD resampling) may be placed as this grid's CTAs finish; it
   // waits for this grid to complete before it touches anything this grid uses.
   cudaTriggerProgrammaticLaunchCompletion();
+  // A chained second stage tests the first stage's tokens (written by the
+  // finish pass two kernels back): those are read only after the wait for the
+  // statistics sweep, whose completion implies that pass's.
+  if (fw.len) cudaGridDependencySynchronize();
 
   // ---- inputs of this call (independent of the statistics kernel) ----
   const float Tf = __ldg(temperature + b);
@@ -842,48 +1011,64 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
     Sd = __ldcg(&si->Sd);
   } else {
     // ---- combine the V-split partials of every row of the window (fp64) ----
-    // Warp w takes rows w, w + NWARP, ...  The partials of a row are those of
-    // the CTAs of the statistics sweep that hold its tiles, in order, CW
-    // consumer warps each.  The first partial per lane of the warp's first two
-    // rows is loaded before either row is reduced, and longer lists (many CTAs
-    // per row, as at B = 1) are read four loads per lane at a time, so the L2
-    // round trips overlap; the order of the fp64 sums is unchanged.
+    // Warp w takes rows w, w + NW, ...  The partials of a row are those of the
+    // CTAs of the statistics sweep that hold its tiles, in order, pcw per CTA
+    // (stored CW apart when pcw = 1).
+    // The first partial per lane of the warp's first two rows is loaded before
+    // either row is reduced, and longer lists (many CTAs per row, as at B = 1)
+    // are read four loads per lane at a time, so the L2 round trips overlap;
+    // the order of the fp64 sums is unchanged.  A partial marked incomplete (a
+    // wait of its sweep CTA ran out) makes the sequence invalid.
     const int RS = fw.srows;  // the sweep's rows per sequence (RW unless only targets)
     auto row_slots = [&](int r) -> int {
       const long long row = b * RS + r;
       return (int)(tile_owner(row * tpr + tpr - 1, G1, tiles) - tile_owner(row * tpr, G1, tiles) +
-                   1) * CW;
+                   1) * pcw;
     };
+    const int pst = pcw == 1 ? CW : 1;  // stride between a row's partials
     Partial pre0, pre1;
     pre0.m = pre1.m = -INFINITY;
     pre0.s = pre1.s = 0.0;
-    if (warp < RS && lane < row_slots(warp)) pre0 = part[(b * RS + warp) * slots * CW + lane];
-    if (warp + NWARP < RS && lane < row_slots(warp + NWARP))
-      pre1 = part[(b * RS + warp + NWARP) * slots * CW + lane];
-    for (int r = warp; r < RS; r += NWARP) {
+    pre0.pad = pre1.pad = 0;
+    if (warp < RS && lane < row_slots(warp)) pre0 = part[(b * RS + warp) * slots * CW + lane * pst];
+    if (warp + NW < RS && lane < row_slots(warp + NW))
+      pre1 = part[(b * RS + warp + NW) * slots * CW + lane * pst];
+    unsigned tmo = 0u;
+    for (int r = warp; r < RS; r += NW) {
       const long long row = b * RS + r;
       const Partial *P = part + row * slots * CW;
       const int nslot = row_slots(r);
       // first 32 partials in registers (one load per lane), the rest streamed
       Partial p0 = r == warp ? pre0 : pre1;
-      if (r >= warp + 2 * NWARP) {
+      if (r >= warp + 2 * NW) {
         p0.m = -INFINITY;
         p0.s = 0.0;
-        if (lane < nslot) p0 = P[lane];
+        p0.pad = 0;
+        if (lane < nslot) p0 = P[lane * pst];
       }
       float m = p0.m;
-#pragma unroll 4
-      for (int s = lane + 32; s < nslot; s += 32) m = fmax_nan(m, P[s].m);
-      m = warp_max_nan(m);
-      double acc =
-          (lane < nslot)
-              ? ((p0.m == -INFINITY) ? p0.s : p0.s * exp2(((double)p0.m - (double)m) * c64))
-              : 0.0;
+      unsigned ab = p0.pad;
 #pragma unroll 4
       for (int s = lane + 32; s < nslot; s += 32) {
-        const Partial ps = P[s];
-        acc += (ps.m == -INFINITY) ? ps.s : ps.s * exp2(((double)ps.m - (double)m) * c64);
+        m = fmax_nan(m, P[s * pst].m);
+        ab |= P[s * pst].pad;
       }
+      m = warp_max_nan(m);
+      tmo |= __any_sync(FULL, ab != 0u) ? 1u : 0u;
+#if SPECDEC_COMBINE_FP32
+      // rescale factors 2^((m_s - m) c) from ex2 (about 2 ulp of fp32)
+      const Scale cs = make_scale(c64);
+      auto rescale = [&](const Partial &ps) -> double {
+        return (ps.m == -INFINITY) ? ps.s : ps.s * (double)ex2(scaled(ps.m - m, cs));
+      };
+#else
+      auto rescale = [&](const Partial &ps) -> double {
+        return (ps.m == -INFINITY) ? ps.s : ps.s * exp2(((double)ps.m - (double)m) * c64);
+      };
+#endif
+      double acc = (lane < nslot) ? rescale(p0) : 0.0;
+#pragma unroll 4
+      for (int s = lane + 32; s < nslot; s += 32) acc += rescale(P[s * pst]);
       acc = warp_sum(acc);
       if (lane == 0) {
         // the row's position and role, and its place in the window's order
@@ -905,6 +1090,7 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
         }
       }
     }
+    if (lane == 0) s_tmo[warp] = tmo;
     if (fw.dstat) {  // the draft rows' statistics, kept by an earlier pass
       for (int i = threadIdx.x; i < fw.np; i += blockDim.x) {
         const Partial *q = fw.dstat + b * (K + 1) + fw.p0 + i;
@@ -916,9 +1102,12 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
 
     // ---- acceptance test and first rejection (warp 0) ----
     if (warp == 0) {
-      // a timed-out wait in this call (or an earlier, unacknowledged one) makes
-      // every sequence invalid rather than silently wrong
-      const bool timed_out = (*(volatile unsigned *)&g_error_flags & SPECDEC_ERR_TIMEOUT) != 0;
+      // a statistics partial left incomplete by a wait that ran out makes the
+      // sequence invalid rather than silently wrong (every CTA of the sequence
+      // reads the same partials, so they all decide alike)
+      unsigned tmo_any = 0u;
+      for (int w = 0; w < NW; ++w) tmo_any |= s_tmo[w];
+      const bool timed_out = tmo_any != 0u;
       bool rows_ok = true;
       for (int r = lane; r < RW; r += 32)
         rows_ok = rows_ok && isfinite(sM[r]) && isfinite(sS[r]) && sS[r] > 0.0;
@@ -963,8 +1152,8 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
           const int tail = nn >= 0 ? nn + 1 : (nn == kChainAll ? m_b : K + 1);
           for (int i = tail + lane; i <= K; i += 32) ot[i] = -1;
           if (lane < m_b && pos <= (nn >= 0 ? nn : K)) {
-            if (dbg_px) dbg_px[b * K + pos] = p;
-            if (dbg_qx) dbg_qx[b * K + pos] = q;
+            if (dbg_px) dbg_px[b * fw.dbg_pstride + pos] = p;
+            if (dbg_qx) dbg_qx[b * fw.dbg_pstride + pos] = q;
           }
         }
         if (lane == 0) {
@@ -975,7 +1164,7 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
             unsigned f = 0;
             if (!t_ok) f |= SPECDEC_ERR_TEMPERATURE;
             if (bad_x) f |= SPECDEC_ERR_TOKEN;
-            if (!rows_ok) f |= SPECDEC_ERR_LOGITS;
+            if (!rows_ok && !timed_out) f |= SPECDEC_ERR_LOGITS;
             atomicOr(&g_error_flags, f);
           }
           if (fw.decide_only && nn >= 0) {  // the drawn pair for the final pass
@@ -1043,8 +1232,9 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
   const int c_beg = cb * cpb;
   const int c_end = (cb + 1) * cpb < nsr ? (cb + 1) * cpb : nsr;
   bool wrote = false;
-  for (int chunk = c_beg + warp; chunk < c_end; chunk += NWARP) {
+  for (int chunk = c_beg + warp; chunk < c_end; chunk += NW) {
     float rs = 0.f;
+    float2 rs2 = make_float2(0.f, 0.f);  // packed partial sums of the vector body
     if (vec_ok) {
       uint4 at[UW], ad[UW];
 #pragma unroll
@@ -1061,7 +1251,9 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
           Dt<T>::unpack(at[k], xt);
           Dt<T>::unpack(ad[k], xd);
 #pragma unroll
-          for (int q = 0; q < VEC; ++q) rs += res_weight(xt[q], xd[q], d);
+          for (int q = 0; q < VEC; q += 2)
+            rs2 = __fadd2_rn(rs2, res_weight2(make_float2(xt[q], xt[q + 1]),
+                                              make_float2(xd[q], xd[q + 1]), d));
         }
       }
       // head elements (chunk 0) and the < VEC tail elements (their chunk)
@@ -1078,7 +1270,7 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
       for (long long v = lo + lane; v < hi; v += 32)
         rs += res_weight(Dt<T>::load(pt + v), d.bonus ? 0.f : Dt<T>::load(pd + v), d);
     }
-    const double tot = warp_sum((double)rs);
+    const double tot = warp_sum((double)rs + ((double)rs2.x + (double)rs2.y));
     if (lane == 0) {
       ResPartial o;
       o.R = tot;
@@ -1102,17 +1294,17 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
   // ---- the last CTA of sequence b draws ----
   __threadfence();
   const ResPartial *rp = rpart + b * nsr;
-  const int cper = (nsr + NT - 1) / NT;  // chunks per thread, contiguous
+  const int cper = (nsr + NTH - 1) / NTH;  // chunks per thread, contiguous
   const int c0 = threadIdx.x * cper < nsr ? threadIdx.x * cper : nsr;
   const int c1 = c0 + cper < nsr ? c0 + cper : nsr;
   double my = 0.0;
   for (int c2 = c0; c2 < c1; ++c2) my += __ldcg(&rp[c2].R);
   double Z;
-  const double cexcl = block_excl_scan(my, Z);
+  const double cexcl = block_excl_scan<NTH>(my, Z);
   if (threadIdx.x == 0) s_mode = (!d.bonus && !(Z >= ldexp(St, -64))) ? 1 : 0;
   __syncthreads();
   if (s_mode == 1) {
-    const int y = draw_exact64(pt, pd, V, d.Mt, St, d.Md, Sd, c64, (double)ures, &s_y, &s_lastpos,
+    const int y = draw_exact64<T, NTH>(pt, pd, V, d.Mt, St, d.Md, Sd, c64, (double)ures, &s_y, &s_lastpos,
                                dbg_Z ? dbg_Z + b : nullptr);
     if (threadIdx.x == 0) out_tokens[b * (K + 1) + n] = y;
     return;
@@ -1157,7 +1349,7 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
   // rescan of the chosen chunk: contiguous elements per thread, in registers
   const long long lo = chunk_lo(s_chunk), hi = chunk_hi(s_chunk);
   const long long L = hi - lo;
-  const long long E = (L + NT - 1) / NT;
+  const long long E = (L + NTH - 1) / NTH;
   const long long e0 = lo + (long long)threadIdx.x * E < hi ? lo + (long long)threadIdx.x * E : hi;
   const long long e1 = (e0 + E < hi) ? e0 + E : hi;
   float w[EMAX];
@@ -1175,7 +1367,7 @@ __global__ void __launch_bounds__(NT, kFinishCtasPerSm) k_finish(
     if (w[k] > 0.0f) lastpos = (int)(e0 + k);
   }
   double ctot;
-  const double excl = block_excl_scan(mysum, ctot);
+  const double excl = block_excl_scan<NTH>(mysum, ctot);
   if (lastpos >= 0) atomicMax(&s_lastpos, lastpos);
   if (s_base >= 0.0) {
     double C = s_base + excl;
@@ -1630,6 +1822,18 @@ __global__ void __launch_bounds__(kTopkThreads, kTopkCtasPerSm) k_topk_exclude(
   }
 }
 
+// the FMA-pipe exponential on its own, for its accuracy test
+__global__ void k_test_exp2(const float *__restrict__ a, float *__restrict__ y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    const float2 r = exp2_fma2(make_float2(a[i], a[i + 1]));
+    y[i] = r.x;
+    y[i + 1] = r.y;
+  } else if (i < n) {
+    y[i] = exp2_fma2(make_float2(a[i], 0.0f)).x;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
@@ -1649,8 +1853,12 @@ struct DeviceBuf {
   void *ptr = nullptr;
   size_t bytes = 0;
 };
-std::unordered_map<int, DeviceBuf> g_ws;       // workspace per device
-std::unordered_map<int, DeviceBuf> g_staging;  // end-to-end staging per device
+// Library-owned buffers, one per (device, stream): calls on different streams
+// may overlap on the GPU, so they must not share partials, chunk sums or
+// arrival tickets.
+using BufKey = std::pair<int, uintptr_t>;
+std::map<BufKey, DeviceBuf> g_ws;       // workspace
+std::map<BufKey, DeviceBuf> g_staging;  // end-to-end staging
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -1659,17 +1867,18 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 struct Sweep {
   int p0, np, bonus, rps;
   int tonly;                  // target rows only (see StatsGeom)
+  int nb;                     // sequences
   long long rows, tiles, G1;  // G1: CTAs of the statistics sweep
   int slots;                  // partial slots per row
 };
 
 struct Plan {
-  int esize, vec, U, tpr, nsr, cpb;
+  int esize, vec, U, tpr, nsr;
   Sweep full;            // the whole batch, every row
   Sweep first, second;   // early exit: positions [0, P), then [P, K] with the bonus row
   Sweep chain;           // chained second stage: the final layer's K+1 rows (the
                          // intermediate's statistics are kept from the first stage)
-  int slots_max;
+  int slots_max;         // partial slots per row in the workspace (the stride of every sweep)
   size_t off_part, off_rpart, off_cnt, off_state, off_info, off_dlogw, off_s1tok, off_s1n,
       off_rstat, total;
 };
@@ -1680,36 +1889,37 @@ int num_sms() {
   return n > 0 ? n : 148;
 }
 
-Sweep make_sweep(int B, int p0, int np, int bonus, int tpr, long long cap);
-
-// A sweep over the target tensor's rows p0 .. p0+np-1 only.
-Sweep make_target_sweep(int B, int p0, int np, int tpr, long long cap) {
-  Sweep w = make_sweep(B, p0, np, 0, tpr, cap);  // (for the partition of np rows per sequence)
-  w.tonly = 1;
-  w.rps = np;
-  w.rows = (long long)B * np;
+// partition of a sweep's tiles over its CTAs and the partial slots per row:
+// the most CTAs whose tile ranges meet one row
+void sweep_partition(Sweep &w, int tpr, long long cap) {
+  w.rows = (long long)w.nb * w.rps;
   w.tiles = w.rows * tpr;
   w.G1 = w.tiles < cap ? w.tiles : cap;
   if (w.G1 < 1) w.G1 = 1;
-  const long long minr = w.tiles / w.G1;
+  const long long minr = w.tiles / w.G1;  // shortest range
   w.slots = minr > 0 ? (int)((tpr - 1 + minr - 1) / minr + 1) : 1;
-  return w;
 }
 
-Sweep make_sweep(int B, int p0, int np, int bonus, int tpr, long long cap) {
+// A sweep over nb sequences: the target and draft rows of positions
+// p0 .. p0+np-1 and, with `bonus`, the target's row K.
+Sweep make_sweep(int nb, int p0, int np, int bonus, int tpr, long long cap) {
   Sweep w;
   w.p0 = p0;
   w.np = np;
   w.bonus = bonus;
   w.rps = 2 * np + bonus;
   w.tonly = 0;
-  w.rows = (long long)B * w.rps;
-  w.tiles = w.rows * tpr;
-  w.G1 = w.tiles < cap ? w.tiles : cap;
-  if (w.G1 < 1) w.G1 = 1;
-  // partial slots per row: the most CTAs whose tile ranges meet one row
-  const long long minr = w.tiles / w.G1;  // shortest range
-  w.slots = minr > 0 ? (int)((tpr - 1 + minr - 1) / minr + 1) : 1;
+  w.nb = nb;
+  sweep_partition(w, tpr, cap);
+  return w;
+}
+
+// A sweep over the target tensor's rows p0 .. p0+np-1 only.
+Sweep make_target_sweep(int nb, int p0, int np, int tpr, long long cap) {
+  Sweep w = make_sweep(nb, p0, np, 0, tpr, cap);
+  w.tonly = 1;
+  w.rps = np;
+  sweep_partition(w, tpr, cap);
   return w;
 }
 
@@ -1748,12 +1958,6 @@ bool make_plan(int B, int K, int V, specdec_dtype dtype, int sms, Plan &pl) {
   // k_finish chunks: 32 lanes x kFinishUW vectors of the drawn row pair
   const long long nr = (nvec_max + 32LL * kFinishUW - 1) / (32LL * kFinishUW);
   pl.nsr = (int)(nr > 0 ? nr : 1);
-  // chunks per CTA of k_finish: as many CTAs per sequence as keep the whole
-  // grid inside one wave (each CTA repeats the small acceptance step)
-  long long ncb = (long long)kFinishCtasPerSm * sms / (B > 0 ? B : 1);
-  if (ncb < 1) ncb = 1;
-  if (ncb > pl.nsr) ncb = pl.nsr;
-  pl.cpb = (int)((pl.nsr + ncb - 1) / ncb);
   if ((long long)B * pl.nsr > INT_MAX) return false;
   if ((long long)B * (K + 1) * (long long)V > (1LL << 56)) return false;
   size_t off = 0;
@@ -1845,6 +2049,12 @@ struct LaunchTimer {
   }
 };
 
+// Test hooks (specdec_test_set_wait_fault): the bound of every on-chip wait,
+// and one tile (local index of a sweep) whose copy the sweep's producer never
+// issues, so that the waits for it run out.
+std::atomic<unsigned long long> g_hook_wait_ns{kWaitNs};
+std::atomic<long long> g_hook_skip_tile{-1};
+
 // Options of one pass (see StatsGeom and FinishWindow).
 struct PassOpts {
   int *state = nullptr;          // early exit: per-sequence decision state
@@ -1855,13 +2065,37 @@ struct PassOpts {
   int d_rows = -1;               // rows per sequence of the draft tensor (default K)
   int tok_stride = -1;           // row stride of tokens and u_accept (default K)
   int emit_count = 0;            // out_n = tokens emitted instead of accepted
+  int dbg_pstride = -1;          // positions per sequence of p_x / q_x (default K)
   Partial *save_t = nullptr;      // keep the target rows' statistics here (see FinishWindow)
   const Partial *dstat = nullptr; // the draft rows' statistics from an earlier pass
 };
 
+template <typename T, int NTH>
+cudaError_t launch_finish(const T *t, const T *d, const int32_t *tok, const float *ua,
+                          const float *ur, const float *temp, int K, int V, const Plan &pl,
+                          const Sweep &sw, int pcw, int ctas_per_sm, bool decide_only, int d_rows,
+                          int tok_stride, const FinishWindow &fw, const Partial *part,
+                          ResPartial *rp, unsigned *cnt, const specdec_debug *dbg,
+                          int32_t *out_tokens, int32_t *out_n, cudaStream_t st) {
+  // CTAs per sequence: as many as keep the grid inside one wave of
+  // ctas_per_sm CTAs per SM (each CTA repeats the small acceptance step); a
+  // decide-only pass draws nothing: one CTA per sequence
+  long long ncb = (long long)ctas_per_sm * num_sms() / (sw.nb > 0 ? sw.nb : 1);
+  if (ncb < 1) ncb = 1;
+  if (ncb > pl.nsr) ncb = pl.nsr;
+  const int cpb = decide_only ? pl.nsr : (int)((pl.nsr + ncb - 1) / ncb);
+  const unsigned g2 = (unsigned)((long long)sw.nb * ((pl.nsr + cpb - 1) / cpb));
+  auto kern = k_finish<T, kFinishUW, NTH>;
+  return launch_pdl(kern, g2, NTH, 0, st, t, d, tok, ua, ur, temp, K, (long long)V, pl.tpr, sw.tiles, sw.G1, pl.slots_max, pcw, pl.nsr, cpb, d_rows, tok_stride, fw,
+                    part, rp, cnt, out_tokens, out_n, dbg ? dbg->row_max : nullptr,
+                    dbg ? dbg->row_sum : nullptr, dbg ? dbg->p_x : nullptr,
+                    dbg ? dbg->q_x : nullptr, dbg ? dbg->Z : nullptr);
+}
+
 // One pass: a statistics sweep over `sw` (of the open sequences when `state`
 // is set and the pass is not the first), then k_finish over the same window
-// (programmatic dependent launch: its launch and gathers overlap the sweep).
+// and sequences (programmatic dependent launch: its launch and gathers overlap
+// the sweep).
 template <typename T>
 specdec_status launch_pass(const void *tg, const void *dr, const int32_t *tok, const float *ua,
                            const float *ur, const float *temp, int B, int K, int V,
@@ -1880,13 +2114,19 @@ specdec_status launch_pass(const void *tg, const void *dr, const int32_t *tok, c
   g.V = V;
   g.tpr = pl.tpr;
   g.tiles = sw.tiles;
-  g.slots = sw.slots;
+  g.slots = pl.slots_max;
   g.p0 = sw.p0;
   g.np = sw.np;
   g.rps = sw.rps;
   g.state = o.decide_only ? nullptr : o.state;  // the first pass reads every sequence
   g.d_rows = d_rows;
   g.tonly = sw.tonly;
+  g.wait_ns = g_hook_wait_ns.load();
+  g.skip_tile = g_hook_skip_tile.load();
+  g.nb = sw.nb;
+  // per-CTA partials where many CTAs share a row (small batches): the finish
+  // pass then reads fewer; otherwise one per warp and no CTA barrier
+  g.pcw = sw.slots > kCtaCombineSlots ? 1 : CW;
   cudaError_t e = cudaSuccess;
   {
     LaunchTimer lt(KID_STATS, st);
@@ -1900,9 +2140,6 @@ specdec_status launch_pass(const void *tg, const void *dr, const int32_t *tok, c
   if (e != cudaSuccess) return SPECDEC_ECUDA;
   {
     LaunchTimer lt(KID_FINISH, st);
-    // a decide-only pass draws nothing: one CTA per sequence
-    const int cpb = o.decide_only ? pl.nsr : pl.cpb;
-    const unsigned g2 = (unsigned)((long long)B * ((pl.nsr + cpb - 1) / cpb));
     FinishWindow fw;
     fw.p0 = sw.p0;
     fw.np = sw.np;
@@ -1917,12 +2154,10 @@ specdec_status launch_pass(const void *tg, const void *dr, const int32_t *tok, c
     fw.dlogw = o.dlogw;
     fw.len = o.len;
     fw.emit_count = o.emit_count;
-    auto kern = k_finish<T, kFinishUW>;
-    e = launch_pdl(kern, g2, NT, 0, st, t, d, tok, ua, ur, temp, K, (long long)V, pl.tpr, sw.tiles,
-                   sw.G1, sw.slots, pl.nsr, cpb, d_rows, tok_stride, fw, (const Partial *)part, rp,
-                   cnt, out_tokens, out_n, dbg ? dbg->row_max : nullptr,
-                   dbg ? dbg->row_sum : nullptr, dbg ? dbg->p_x : nullptr,
-                   dbg ? dbg->q_x : nullptr, dbg ? dbg->Z : nullptr);
+    fw.dbg_pstride = o.dbg_pstride > 0 ? o.dbg_pstride : K;
+    e = launch_finish<T, kFinishThreads>(t, d, tok, ua, ur, temp, K, V, pl, sw, g.pcw,
+                                         kFinishCtasPerSm, o.decide_only, d_rows, tok_stride, fw,
+                                         part, rp, cnt, dbg, out_tokens, out_n, st);
   }
   return e == cudaSuccess ? SPECDEC_OK : SPECDEC_ECUDA;
 }
@@ -1957,7 +2192,7 @@ specdec_status launch_chained(const void *fin, const void *inter, const void *dr
                               const float *ua2, const float *ur2, const float *temp, int B,
                               int K, int V, const Plan &pl, char *ws, int32_t *s1_tok,
                               int32_t *s1_n, int32_t *out_tokens, int32_t *out_emitted,
-                              cudaStream_t st) {
+                              const specdec_debug *dbg2, cudaStream_t st) {
   Partial *rstat = reinterpret_cast<Partial *>(ws + pl.off_rstat);
   PassOpts o1;
   o1.save_t = rstat;  // the intermediate rows' statistics, for the second stage
@@ -1970,8 +2205,9 @@ specdec_status launch_chained(const void *fin, const void *inter, const void *dr
   o.tok_stride = K + 1;
   o.emit_count = 1;
   o.dstat = rstat;  // the second stage sweeps the final layer's rows only
+  o.dbg_pstride = K + 1;
   return launch_pass<T>(fin, inter, s1_tok, ua2, ur2, temp, B, K, V, pl, pl.chain, o, ws,
-                        nullptr, out_tokens, out_emitted, st);
+                        dbg2, out_tokens, out_emitted, st);
 }
 
 specdec_status check_args(const void *tg, const void *dr, const int32_t *tok, const float *ua,
@@ -2059,13 +2295,14 @@ specdec_status run_smc(const void *tg, const void *dr, const int32_t *tok, const
   return e == cudaSuccess ? SPECDEC_OK : SPECDEC_ECUDA;
 }
 
-// grow-only device buffer of the current device (zero-filled when (re)allocated)
-specdec_status ensure_buf(std::unordered_map<int, DeviceBuf> &map, size_t bytes,
-                          cudaStream_t st, void **out) {
+// grow-only device buffer of the current device and this stream (zero-filled
+// when (re)allocated)
+specdec_status ensure_buf(std::map<BufKey, DeviceBuf> &map, size_t bytes, cudaStream_t st,
+                          void **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SPECDEC_ECUDA;
   std::lock_guard<std::mutex> lk(g_mu);
-  DeviceBuf &db = map[dev];
+  DeviceBuf &db = map[BufKey(dev, reinterpret_cast<uintptr_t>(st))];
   if (db.bytes < bytes) {
     cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
     if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return SPECDEC_ECUDA;
@@ -2243,12 +2480,13 @@ specdec_status specdec_topk_exclude(const void *logits, long long row_stride,
   return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ECUDA;
 }
 
-specdec_status specdec_verify_chained(
+specdec_status specdec_verify_chained_ex(
     const void *final_logits, const void *intermediate_logits, const void *draft_logits,
     const int32_t *draft_tokens, const float *u_accept1, const float *u_resample1,
     const float *u_accept2, const float *u_resample2, const float *temperature, int B, int K,
     int V, specdec_dtype dtype, int32_t *out_tokens, int32_t *out_num_emitted,
-    int32_t *stage1_tokens, int32_t *stage1_num_accepted, void *stream) {
+    int32_t *stage1_tokens, int32_t *stage1_num_accepted, const specdec_debug *dbg2,
+    void *stream) {
   if (K > 31) return SPECDEC_EINVAL;  // the second stage tests K+1 positions on one warp
   specdec_status s = check_args(intermediate_logits, draft_logits, draft_tokens, u_accept1,
                                 u_resample1, temperature, B, K, V, dtype, out_tokens,
@@ -2275,10 +2513,22 @@ specdec_status specdec_verify_chained(
     return launch_chained<__nv_bfloat16>(final_logits, intermediate_logits, draft_logits,
                                          draft_tokens, u_accept1, u_resample1, u_accept2,
                                          u_resample2, temperature, B, K, V, pl, w, s1t, s1n,
-                                         out_tokens, out_num_emitted, st);
+                                         out_tokens, out_num_emitted, dbg2, st);
   return launch_chained<float>(final_logits, intermediate_logits, draft_logits, draft_tokens,
                                u_accept1, u_resample1, u_accept2, u_resample2, temperature, B,
-                               K, V, pl, w, s1t, s1n, out_tokens, out_num_emitted, st);
+                               K, V, pl, w, s1t, s1n, out_tokens, out_num_emitted, dbg2, st);
+}
+
+specdec_status specdec_verify_chained(
+    const void *final_logits, const void *intermediate_logits, const void *draft_logits,
+    const int32_t *draft_tokens, const float *u_accept1, const float *u_resample1,
+    const float *u_accept2, const float *u_resample2, const float *temperature, int B, int K,
+    int V, specdec_dtype dtype, int32_t *out_tokens, int32_t *out_num_emitted,
+    int32_t *stage1_tokens, int32_t *stage1_num_accepted, void *stream) {
+  return specdec_verify_chained_ex(final_logits, intermediate_logits, draft_logits, draft_tokens,
+                                   u_accept1, u_resample1, u_accept2, u_resample2, temperature,
+                                   B, K, V, dtype, out_tokens, out_num_emitted, stage1_tokens,
+                                   stage1_num_accepted, nullptr, stream);
 }
 
 specdec_status specdec_verify_bf16(const void *target_logits, const void *draft_logits,
@@ -2383,7 +2633,7 @@ void specdec_release(void) {
   for (auto *m : {&g_ws, &g_staging}) {
     for (auto &kv : *m) {
       if (kv.second.ptr) {
-        cudaSetDevice(kv.first);
+        cudaSetDevice(kv.first.first);
         cudaDeviceSynchronize();
         cudaFree(kv.second.ptr);
       }
@@ -2391,6 +2641,32 @@ void specdec_release(void) {
     m->clear();
   }
   cudaSetDevice(cur);
+}
+
+specdec_status specdec_get_error(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return SPECDEC_ECUDA;
+  unsigned v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_error_flags, sizeof v) != cudaSuccess) return SPECDEC_ECUDA;
+  if (cudaMemcpyToSymbol(g_error_flags, &zero, sizeof zero) != cudaSuccess) return SPECDEC_ECUDA;
+  return v ? SPECDEC_EDEVICE : SPECDEC_OK;
+}
+
+const char *specdec_error_string(specdec_status s) { return specdec_status_string(s); }
+
+specdec_status specdec_test_exp2(const float *a, float *y, int n, void *stream) {
+  if (n < 0 || (n > 0 && (!a || !y))) return SPECDEC_EINVAL;
+  if (n == 0) return SPECDEC_OK;
+  const int threads = 256;
+  const int blocks = (int)(((long long)(n + 1) / 2 + threads - 1) / threads);
+  k_test_exp2<<<blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(a, y, n);
+  return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ECUDA;
+}
+
+specdec_status specdec_test_set_wait_fault(long long skip_tile, unsigned long long wait_ns) {
+  if (skip_tile < -1 || wait_ns == 0) return SPECDEC_EINVAL;
+  g_hook_skip_tile.store(skip_tile);
+  g_hook_wait_ns.store(wait_ns);
+  return SPECDEC_OK;
 }
 
 const char *specdec_status_string(specdec_status s) {

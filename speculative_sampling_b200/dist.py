@@ -24,14 +24,16 @@ def shard_range(per_rank: int, rank: int) -> Tuple[int, int]:
     return rank * per_rank, (rank + 1) * per_rank
 
 
-def generate_shard(workload: str, rank: int, world: int, per_rank: int = None):
+def generate_shard(workload: str, rank: int, world: int, per_rank: int = None,
+                   sigma: float = None):
     """This rank's inputs: sequences [rank*B, (rank+1)*B) of a batch of
-    world*B sequences of ``workload`` (B = the workload's batch by default).
-    Equal, array for array, to the same slice of the whole batch."""
+    world*B sequences of ``workload`` (B = the workload's batch by default;
+    ``sigma`` overrides its draft noise).  Equal, array for array, to the same
+    slice of the whole batch."""
     w = _inputs.WORKLOADS[workload]
     B = w.B if per_rank is None else per_rank
     b0, b1 = shard_range(B, rank)
-    return _inputs.generate(workload, seq_begin=b0, seq_end=b1, B=B * world)
+    return _inputs.generate(workload, seq_begin=b0, seq_end=b1, B=B * world, sigma=sigma)
 
 
 def max_over_ranks(value: float, device=None) -> float:
