@@ -333,6 +333,10 @@ __device__ __forceinline__ float2 exp2_fma2(float2 a) {
   return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
                      __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
+// 1: the sweep's exponent arguments with log2(e)/T as one fp32 value
+#ifndef SPECDEC_SINGLE_SCALE
+#define SPECDEC_SINGLE_SCALE 0
+#endif
 // pairs of each 16-byte vector whose exponentials the sweep takes on the FMA
 // pipe (the rest on MUFU)
 #ifndef SPECDEC_EXP_FMA_PAIRS
@@ -410,7 +414,11 @@ __device__ __forceinline__ void vec_fold(const uint4 &v, RunStat &q, Scale c, fl
 #pragma unroll
   for (int k = 0; k < N; ++k) {
     const float2 d = __fadd2_rn(x[k], nr);
+#if SPECDEC_SINGLE_SCALE
+    const float2 a = __fmul2_rn(d, __fadd2_rn(hi, lo));
+#else
     const float2 a = __ffma2_rn(d, hi, __fmul2_rn(d, lo));
+#endif
     if (k < SPECDEC_EXP_FMA_PAIRS)
       e[k] = exp2_fma2(a);
     else
@@ -776,22 +784,10 @@ struct DrawRow {
 // r = St * max(0, p - q) = max(0, e_t - (St/Sd) e_d) with e = 2^((z - m)c)
 // (or e_t for the bonus row).  The same inlined arithmetic serves the chunk
 // sums and the rescan, so both see bit-identical per-element weights.
-#ifndef SPECDEC_FINISH_EXP_FMA
-#define SPECDEC_FINISH_EXP_FMA 0
-#endif
-#ifndef SPECDEC_COMBINE_FP32
-#define SPECDEC_COMBINE_FP32 0
-#endif
 __device__ __forceinline__ float res_weight(float zt, float zd, const DrawRow &d) {
   const float et = ex2(scaled(zt - d.Mt, d.c));
   if (d.bonus) return et;
-#if SPECDEC_FINISH_EXP_FMA
-  // the draft row's exponential on the FMA pipe (the MUFU unit takes the
-  // target's): the finish pass is MUFU-bound
-  const float ed = exp2_fma2(make_float2(scaled(zd - d.Md, d.c), -125.0f)).x;
-#else
   const float ed = ex2(scaled(zd - d.Md, d.c));
-#endif
   const float t1 = __fmaf_rn(-d.lhi, ed, et);
   const float t2 = __fmaf_rn(-d.llo, ed, t1);
   return t2 > 0.0f ? t2 : 0.0f;
@@ -807,11 +803,7 @@ __device__ __forceinline__ float2 res_weight2(float2 zt, float2 zd, const DrawRo
   if (d.bonus) return et;
   const float2 dd = __fadd2_rn(zd, make_float2(-d.Md, -d.Md));
   const float2 ad = __ffma2_rn(dd, hi, __fmul2_rn(dd, lo));
-#if SPECDEC_FINISH_EXP_FMA
-  const float2 ed = exp2_fma2(ad);
-#else
   const float2 ed = make_float2(ex2(ad.x), ex2(ad.y));
-#endif
   const float2 t1 = __ffma2_rn(make_float2(-d.lhi, -d.lhi), ed, et);
   const float2 t2 = __ffma2_rn(make_float2(-d.llo, -d.llo), ed, t1);
   return make_float2(t2.x > 0.0f ? t2.x : 0.0f, t2.y > 0.0f ? t2.y : 0.0f);
@@ -1046,29 +1038,35 @@ __global__ void __launch_bounds__(NTH, 65536 / (NTH * kFinishMaxNreg)) k_finish(
         p0.pad = 0;
         if (lane < nslot) p0 = P[lane * pst];
       }
-      float m = p0.m;
-      unsigned ab = p0.pad;
+      // the lane's next three partials in registers too (one round of loads);
+      // rows with more than 128 partials read the rest in a loop
+      Partial px[3];
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+        px[k].m = -INFINITY;
+        px[k].s = 0.0;
+        px[k].pad = 0;
+        const int sk = lane + 32 * (k + 1);
+        if (sk < nslot) px[k] = P[sk * pst];
+      }
+      float m = fmax_nan(fmax3_nan(p0.m, px[0].m, px[1].m), px[2].m);
+      unsigned ab = p0.pad | px[0].pad | px[1].pad | px[2].pad;
 #pragma unroll 4
-      for (int s = lane + 32; s < nslot; s += 32) {
+      for (int s = lane + 128; s < nslot; s += 32) {
         m = fmax_nan(m, P[s * pst].m);
         ab |= P[s * pst].pad;
       }
       m = warp_max_nan(m);
       tmo |= __any_sync(FULL, ab != 0u) ? 1u : 0u;
-#if SPECDEC_COMBINE_FP32
-      // rescale factors 2^((m_s - m) c) from ex2 (about 2 ulp of fp32)
-      const Scale cs = make_scale(c64);
-      auto rescale = [&](const Partial &ps) -> double {
-        return (ps.m == -INFINITY) ? ps.s : ps.s * (double)ex2(scaled(ps.m - m, cs));
-      };
-#else
       auto rescale = [&](const Partial &ps) -> double {
         return (ps.m == -INFINITY) ? ps.s : ps.s * exp2(((double)ps.m - (double)m) * c64);
       };
-#endif
       double acc = (lane < nslot) ? rescale(p0) : 0.0;
+#pragma unroll
+      for (int k = 0; k < 3; ++k)
+        if (lane + 32 * (k + 1) < nslot) acc += rescale(px[k]);
 #pragma unroll 4
-      for (int s = lane + 32; s < nslot; s += 32) acc += rescale(P[s * pst]);
+      for (int s = lane + 128; s < nslot; s += 32) acc += rescale(P[s * pst]);
       acc = warp_sum(acc);
       if (lane == 0) {
         // the row's position and role, and its place in the window's order
@@ -1529,19 +1527,18 @@ __global__ void __launch_bounds__(NT) k_smc_resample(const double *__restrict__ 
 // row other than x_{i+1} are the candidates for the next-next token.  Order:
 // larger logit first, equal logits by ascending token id; a row with a NaN is
 // invalid.  One CTA per row:
-//   1. one pass: each thread's running max of an order-preserving key of the
-//      logits (and a NaN check).  The k-th largest of the 256 thread maxima,
-//      tau0, is at most the row's k-th largest key (k distinct elements reach
-//      it), so every answer has key >= tau0;
+//   1. the thread maxima of the row give a lower bound tau of its k-th
+//      largest key (radix select on the top 16 key bits);
 //   2. a second pass (from L2) appends every non-excluded element with
-//      key >= tau0 to a shared buffer (about k of them for real logits);
-//      a bitonic sort of (key, ~index) gives the order;
-//   3. when ties at the top overflow the buffer (e.g. a constant row), an
-//      exact radix select of the k-th key (8 bits per pass) and an
-//      index-ordered pick among the keys equal to it replace step 2.
+//      key >= tau to a shared buffer (about k of them for real logits) and
+//      checks for NaN;
+//   3. each candidate's rank (the number of candidates above it) places it;
+//      up to the buffer's size a bitonic sort of (key, ~index) does it
+//      instead, and when ties at the top overflow the buffer (e.g. a constant
+//      row) an exact radix select of the k-th key (8 bits per pass) and an
+//      index-ordered pick among the keys equal to it take over.
 // 512 threads per row, three CTAs per SM (all 320 rows of a B=64, K=5 batch
-// resident at once): more loads in flight than 256 threads, and a tighter
-// threshold (the k-th largest of 512 thread maxima)
+// resident at once).
 constexpr int kTopkThreads = 512;
 constexpr int kTopkCtasPerSm = 3;
 constexpr int kTopkMaxK = 256;
@@ -1663,7 +1660,6 @@ __global__ void __launch_bounds__(kTopkThreads, kTopkCtasPerSm) k_topk_exclude(
     int V, const int32_t *__restrict__ exclude, int k, int32_t *__restrict__ out_idx,
     float *__restrict__ out_val) {
   __shared__ unsigned long long cand[kTopkCap];  // (key << 32) | ~index
-  __shared__ uint32_t tmax[kTopkThreads];
   __shared__ unsigned hist[256];
   __shared__ int s_n, s_bad, s_rem, s_cnt[kTopkThreads / 32];
   __shared__ uint32_t s_prefix;
@@ -1679,33 +1675,117 @@ __global__ void __launch_bounds__(kTopkThreads, kTopkCtasPerSm) k_topk_exclude(
     s_n = 0;
     s_bad = 0;
   }
-  // 1. thread maxima (and NaN check): a packed max per vector; only the
-  // vector holding the excluded token is unpacked
+  // 1. A lower bound tau of the row's k-th largest key: the thread maxima of
+  // the row are distinct elements, so their k-th largest is at most the
+  // row's.  It is found by a radix select on the top 16 key bits (two 8-bit
+  // histogram passes), and tau is the smallest key of its 16-bit bucket
+  // (exact for bf16 keys).  NaNs are left out here; the second pass finds
+  // them.
   constexpr int VEC = Dt<T>::VEC;
+  const int head = row_head(row, (long long)V);
+  const int nvec = (V - head) / VEC;
+  const int P = nvec;
+  const uint4 *pv = reinterpret_cast<const uint4 *>(row + head);
   float mx = -INFINITY;
-  bool bad = false, seen = false;
-  auto scalar1 = [&](int v, float x) {
-    bad |= isnan(x);
-    if (v != ex) {
-      mx = fmax_nan(mx, x);
+  bool seen = false;
+  auto take1 = [&](int v, float x) {
+    if (v != ex && !isnan(x)) {
+      mx = fmaxf(mx, x);
       seen = true;
     }
   };
+  if (tid < head) take1(tid, Dt<T>::load(row + tid));
+  for (int i0 = tid; i0 < P; i0 += 4 * kTopkThreads) {
+    uint4 w[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * kTopkThreads;
+      w[u] = i < P ? __ldg(pv + i) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * kTopkThreads;
+      if (i >= P) continue;
+      const int v0 = head + i * VEC;
+      const float m = vec_max_nan<T>(w[u]);
+      if (ex >= v0 && ex < v0 + VEC || isnan(m)) {
+        float x[VEC];
+        Dt<T>::unpack(w[u], x);
+#pragma unroll
+        for (int e2 = 0; e2 < VEC; ++e2) take1(v0 + e2, x[e2]);
+      } else {
+        mx = fmaxf(mx, m);
+        seen = true;
+      }
+    }
+  }
+  const uint32_t tkey = seen ? logit_key(mx) : 0u;  // 0: no value (below every key)
+  uint32_t prefix = 0;
+  int rem = k;
+  for (int shift = 24; shift >= 16; shift -= 8) {
+    for (int i = tid; i < 256; i += kTopkThreads) hist[i] = 0;
+    __syncthreads();
+    if (shift == 24 || (tkey >> 24) == (prefix >> 24)) atomicAdd(&hist[(tkey >> shift) & 255u], 1u);
+    __syncthreads();
+    if (warp == 0) {
+      // lane l holds buckets 255 - 8l - j, j < 8 (from the top); find the
+      // bucket where the count from the top reaches rem
+      unsigned c8 = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) c8 += hist[255 - 8 * lane - j];
+      unsigned incl = c8;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(FULL, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const unsigned excl = incl - c8;
+      const bool here = excl < (unsigned)rem && incl >= (unsigned)rem;
+      const unsigned who = __ballot_sync(FULL, here);
+      if (who != 0u && lane == __ffs(who) - 1) {
+        unsigned cum = excl;
+        int d = 255 - 8 * lane;
+        for (int j = 0; j < 8; ++j, --d) {
+          if (cum + hist[d] >= (unsigned)rem) break;
+          cum += hist[d];
+        }
+        s_rem = rem - (int)cum;
+        s_prefix = prefix | ((uint32_t)d << shift);
+      } else if (who == 0u && lane == 0) {  // fewer than rem keys in all: every key qualifies
+        s_rem = rem;
+        s_prefix = prefix;
+      }
+    }
+    __syncthreads();
+    prefix = s_prefix;
+    rem = s_rem;
+    __syncthreads();
+  }
+  const uint32_t tau = prefix;  // the bucket's smallest key (low 16 bits 0)
+  // 2. A second pass over the row (now in L2): every non-excluded key >= tau
+  // goes to the candidate buffer (a vector is unpacked only when its max
+  // reaches tau or is NaN); a NaN anywhere makes the row invalid.
+  bool bad = false;
+  auto scalar2 = [&](int v, float x) {
+    bad |= isnan(x);
+    const uint32_t key = logit_key(x);
+    if (v != ex && key >= tau && !isnan(x)) {
+      const int pos = atomicAdd(&s_n, 1);
+      if (pos < kTopkCap)
+        cand[pos] = ((unsigned long long)key << 32) | (unsigned)(0xFFFFFFFFu - (unsigned)v);
+    }
+  };
   row_foreach_vec(row, V, [&](int v0, const uint4 &w) {
-    if (ex >= v0 && ex < v0 + VEC) {
+    const float m = vec_max_nan<T>(w);
+    if (isnan(m) || logit_key(m) >= tau) {
       float x[VEC];
       Dt<T>::unpack(w, x);
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) scalar1(v0 + e, x[e]);
-    } else {
-      mx = fmax_nan(mx, vec_max_nan<T>(w));
-      seen = true;
+      for (int e2 = 0; e2 < VEC; ++e2) scalar2(v0 + e2, x[e2]);
     }
-  }, scalar1);
-  bad |= isnan(mx);
-  tmax[tid] = (seen && !isnan(mx)) ? logit_key(mx) : 0u;
+  }, scalar2);
   if (__any_sync(FULL, bad) && lane == 0) s_bad = 1;
-  bitonic_desc(tmax, kTopkThreads);
+  __syncthreads();
   if (s_bad) {  // invalid row
     for (int i = tid; i < k; i += blockDim.x) {
       oi[i] = -1;
@@ -1714,27 +1794,27 @@ __global__ void __launch_bounds__(kTopkThreads, kTopkCtasPerSm) k_topk_exclude(
     if (tid == 0) atomicOr(&g_error_flags, SPECDEC_ERR_LOGITS);
     return;
   }
-  const uint32_t tau0 = tmax[k - 1];  // 0 when fewer than k threads saw a value
-  // 2. candidates: every non-excluded key >= tau0 (a vector is unpacked only
-  // when its max reaches tau0)
-  auto scalar2 = [&](int v, float x) {
-    const uint32_t key = logit_key(x);
-    if (v != ex && key >= tau0) {
-      const int pos = atomicAdd(&s_n, 1);
-      if (pos < kTopkCap)
-        cand[pos] = ((unsigned long long)key << 32) | (unsigned)(0xFFFFFFFFu - (unsigned)v);
-    }
-  };
-  row_foreach_vec(row, V, [&](int v0, const uint4 &w) {
-    if (logit_key(vec_max_nan<T>(w)) >= tau0) {
-      float x[VEC];
-      Dt<T>::unpack(w, x);
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) scalar2(v0 + e, x[e]);
-    }
-  }, scalar2);
-  __syncthreads();
   int n = s_n;
+  if (n <= 2 * kTopkThreads) {
+    // 3. few candidates (about k for real logits): each one's place in the
+    // order is the number of candidates above it ((key, ~index) pairs are
+    // unique); no sort
+    for (int i = tid; i < n; i += kTopkThreads) {
+      const unsigned long long c = cand[i];
+      int rank = 0;
+      for (int j = 0; j < n; ++j) rank += cand[j] > c ? 1 : 0;
+      if (rank < k) {
+        const int v = (int)(0xFFFFFFFFu - (unsigned)(c & 0xFFFFFFFFull));
+        oi[rank] = v;
+        if (ov) ov[rank] = Dt<T>::load(row + v);
+      }
+    }
+    for (int i = n + tid; i < k; i += blockDim.x) {
+      oi[i] = -1;
+      if (ov) ov[i] = -INFINITY;
+    }
+    return;
+  }
   if (n > kTopkCap) {
     // 3. ties overflowed the buffer: exact k-th key by radix select
     const int KB = sizeof(T) == 2 ? 16 : 32;  // bf16 keys live in the top 16 bits
