@@ -169,6 +169,17 @@ __device__ __forceinline__ float warp_max_nan(float v) {
   for (int o = 16; o; o >>= 1) v = fmax_nan(v, __shfl_xor_sync(FULL, v, o));
   return v;
 }
+// reductions within each 16-lane half of a warp (all 32 lanes call them)
+__device__ __forceinline__ double half_sum(double v) {
+#pragma unroll
+  for (int o = 8; o; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
+  return v;
+}
+__device__ __forceinline__ float half_max_nan(float v) {
+#pragma unroll
+  for (int o = 8; o; o >>= 1) v = fmax_nan(v, __shfl_xor_sync(FULL, v, o));
+  return v;
+}
 
 // ---------------------------------------------------------------------------
 // kernel 1: softmax statistics of every row
@@ -947,7 +958,7 @@ __global__ void __launch_bounds__(NTH, 65536 / (NTH * kFinishMaxNreg)) k_finish(
   __shared__ float sM[66];
   __shared__ double sS[66];
   __shared__ int s_n, s_last, s_mode, s_chunk, s_y, s_lastpos;
-  __shared__ unsigned s_tmo[NW];  // per warp: a partial it read was marked incomplete
+  __shared__ unsigned s_tmo[2 * NW];  // per half-warp: a partial it read was marked incomplete
   __shared__ double s_base, s_t;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int ncb = (nsr + cpb - 1) / cpb;  // CTAs per sequence
@@ -1003,14 +1014,13 @@ __global__ void __launch_bounds__(NTH, 65536 / (NTH * kFinishMaxNreg)) k_finish(
     Sd = __ldcg(&si->Sd);
   } else {
     // ---- combine the V-split partials of every row of the window (fp64) ----
-    // Warp w takes rows w, w + NW, ...  The partials of a row are those of the
+    // Half-warp h (16 lanes) takes rows h, h + 2*NW, ..., so a window of up to
+    // 2*NW rows is reduced in one step.  The partials of a row are those of the
     // CTAs of the statistics sweep that hold its tiles, in order, pcw per CTA
-    // (stored CW apart when pcw = 1).
-    // The first partial per lane of the warp's first two rows is loaded before
-    // either row is reduced, and longer lists (many CTAs per row, as at B = 1)
-    // are read four loads per lane at a time, so the L2 round trips overlap;
-    // the order of the fp64 sums is unchanged.  A partial marked incomplete (a
-    // wait of its sweep CTA ran out) makes the sequence invalid.
+    // (stored CW apart when pcw = 1); a lane loads up to four of them in one
+    // round (longer lists, as at B = 1, are read in a loop), so the L2 round
+    // trips overlap.  A partial marked incomplete (a wait of its sweep CTA ran
+    // out) makes the sequence invalid.
     const int RS = fw.srows;  // the sweep's rows per sequence (RW unless only targets)
     auto row_slots = [&](int r) -> int {
       const long long row = b * RS + r;
@@ -1018,57 +1028,43 @@ __global__ void __launch_bounds__(NTH, 65536 / (NTH * kFinishMaxNreg)) k_finish(
                    1) * pcw;
     };
     const int pst = pcw == 1 ? CW : 1;  // stride between a row's partials
-    Partial pre0, pre1;
-    pre0.m = pre1.m = -INFINITY;
-    pre0.s = pre1.s = 0.0;
-    pre0.pad = pre1.pad = 0;
-    if (warp < RS && lane < row_slots(warp)) pre0 = part[(b * RS + warp) * slots * CW + lane * pst];
-    if (warp + NW < RS && lane < row_slots(warp + NW))
-      pre1 = part[(b * RS + warp + NW) * slots * CW + lane * pst];
+    const int hw = threadIdx.x >> 4, hl = lane & 15;
+    const unsigned hmask = 0xFFFFu << (lane & 16);
     unsigned tmo = 0u;
-    for (int r = warp; r < RS; r += NW) {
-      const long long row = b * RS + r;
-      const Partial *P = part + row * slots * CW;
-      const int nslot = row_slots(r);
-      // first 32 partials in registers (one load per lane), the rest streamed
-      Partial p0 = r == warp ? pre0 : pre1;
-      if (r >= warp + 2 * NW) {
-        p0.m = -INFINITY;
-        p0.s = 0.0;
-        p0.pad = 0;
-        if (lane < nslot) p0 = P[lane * pst];
-      }
-      // the lane's next three partials in registers too (one round of loads);
-      // rows with more than 128 partials read the rest in a loop
-      Partial px[3];
+    for (int r0 = 0; r0 < RS; r0 += 2 * NW) {
+      const int r = r0 + hw;
+      const bool has = r < RS;
+      const Partial *P = part + (b * RS + (has ? r : 0)) * slots * CW;
+      const int nslot = has ? row_slots(r) : 0;
+      Partial px[4];
 #pragma unroll
-      for (int k = 0; k < 3; ++k) {
+      for (int k = 0; k < 4; ++k) {
         px[k].m = -INFINITY;
         px[k].s = 0.0;
         px[k].pad = 0;
-        const int sk = lane + 32 * (k + 1);
+        const int sk = hl + 16 * k;
         if (sk < nslot) px[k] = P[sk * pst];
       }
-      float m = fmax_nan(fmax3_nan(p0.m, px[0].m, px[1].m), px[2].m);
-      unsigned ab = p0.pad | px[0].pad | px[1].pad | px[2].pad;
+      float m = fmax_nan(fmax3_nan(px[0].m, px[1].m, px[2].m), px[3].m);
+      unsigned ab = px[0].pad | px[1].pad | px[2].pad | px[3].pad;
 #pragma unroll 4
-      for (int s = lane + 128; s < nslot; s += 32) {
+      for (int s = hl + 64; s < nslot; s += 16) {
         m = fmax_nan(m, P[s * pst].m);
         ab |= P[s * pst].pad;
       }
-      m = warp_max_nan(m);
-      tmo |= __any_sync(FULL, ab != 0u) ? 1u : 0u;
+      m = half_max_nan(m);
+      tmo |= (__ballot_sync(FULL, ab != 0u) & hmask) ? 1u : 0u;
       auto rescale = [&](const Partial &ps) -> double {
         return (ps.m == -INFINITY) ? ps.s : ps.s * exp2(((double)ps.m - (double)m) * c64);
       };
-      double acc = (lane < nslot) ? rescale(p0) : 0.0;
+      double acc = 0.0;
 #pragma unroll
-      for (int k = 0; k < 3; ++k)
-        if (lane + 32 * (k + 1) < nslot) acc += rescale(px[k]);
+      for (int k = 0; k < 4; ++k)
+        if (hl + 16 * k < nslot) acc += rescale(px[k]);
 #pragma unroll 4
-      for (int s = lane + 128; s < nslot; s += 32) acc += rescale(P[s * pst]);
-      acc = warp_sum(acc);
-      if (lane == 0) {
+      for (int s = hl + 64; s < nslot; s += 16) acc += rescale(P[s * pst]);
+      acc = half_sum(acc);
+      if (has && hl == 0) {
         // the row's position and role, and its place in the window's order
         const bool is_t = fw.dstat || !(r < 2 * fw.np && (r & 1));
         const int rp = fw.dstat ? fw.p0 + r : (r < 2 * fw.np ? fw.p0 + (r >> 1) : K);
@@ -1088,7 +1084,7 @@ __global__ void __launch_bounds__(NTH, 65536 / (NTH * kFinishMaxNreg)) k_finish(
         }
       }
     }
-    if (lane == 0) s_tmo[warp] = tmo;
+    if (hl == 0) s_tmo[hw] = tmo;
     if (fw.dstat) {  // the draft rows' statistics, kept by an earlier pass
       for (int i = threadIdx.x; i < fw.np; i += blockDim.x) {
         const Partial *q = fw.dstat + b * (K + 1) + fw.p0 + i;
@@ -1104,7 +1100,7 @@ __global__ void __launch_bounds__(NTH, 65536 / (NTH * kFinishMaxNreg)) k_finish(
       // sequence invalid rather than silently wrong (every CTA of the sequence
       // reads the same partials, so they all decide alike)
       unsigned tmo_any = 0u;
-      for (int w = 0; w < NW; ++w) tmo_any |= s_tmo[w];
+      for (int w = 0; w < 2 * NW; ++w) tmo_any |= s_tmo[w];
       const bool timed_out = tmo_any != 0u;
       bool rows_ok = true;
       for (int r = lane; r < RW; r += 32)
@@ -1285,6 +1281,7 @@ __global__ void __launch_bounds__(NTH, 65536 / (NTH * kFinishMaxNreg)) k_finish(
     s_chunk = INT_MAX;
     s_y = INT_MAX;
     s_lastpos = -1;
+    s_base = -1.0;  // < 0 selects the "last positive element" rule
   }
   __syncthreads();
   if (!s_last) return;
@@ -1295,8 +1292,17 @@ __global__ void __launch_bounds__(NTH, 65536 / (NTH * kFinishMaxNreg)) k_finish(
   const int cper = (nsr + NTH - 1) / NTH;  // chunks per thread, contiguous
   const int c0 = threadIdx.x * cper < nsr ? threadIdx.x * cper : nsr;
   const int c1 = c0 + cper < nsr ? c0 + cper : nsr;
+  // the thread's chunk sums are read once: the first kDrawRegChunks kept in
+  // registers (every chunk when nsr <= kDrawRegChunks * NTH), later ones re-read
+  constexpr int kDrawRegChunks = 4;
+  double rv[kDrawRegChunks];
   double my = 0.0;
-  for (int c2 = c0; c2 < c1; ++c2) my += __ldcg(&rp[c2].R);
+#pragma unroll
+  for (int k = 0; k < kDrawRegChunks; ++k) {
+    rv[k] = (c0 + k < c1) ? __ldcg(&rp[c0 + k].R) : 0.0;
+    my += rv[k];
+  }
+  for (int c2 = c0 + kDrawRegChunks; c2 < c1; ++c2) my += __ldcg(&rp[c2].R);
   double Z;
   const double cexcl = block_excl_scan<NTH>(my, Z);
   if (threadIdx.x == 0) s_mode = (!d.bonus && !(Z >= ldexp(St, -64))) ? 1 : 0;
@@ -1308,21 +1314,37 @@ __global__ void __launch_bounds__(NTH, 65536 / (NTH * kFinishMaxNreg)) k_finish(
     return;
   }
   const double t = (double)ures * Z;
+  // the chunk holding t: its thread claims it and keeps its exclusive prefix
+  int my_chunk = INT_MAX;
+  double my_base = -1.0;
   {
     double C = cexcl;
-    for (int c2 = c0; c2 < c1; ++c2) {
+#pragma unroll
+    for (int k = 0; k < kDrawRegChunks; ++k) {
+      if (my_chunk == INT_MAX && c0 + k < c1) {
+        if (C <= t && t < C + rv[k]) {
+          my_chunk = c0 + k;
+          my_base = C;
+        }
+        C += rv[k];
+      }
+    }
+    for (int c2 = c0 + kDrawRegChunks; my_chunk == INT_MAX && c2 < c1; ++c2) {
       const double v = __ldcg(&rp[c2].R);
       if (C <= t && t < C + v) {
-        atomicMin(&s_chunk, c2);
-        break;
+        my_chunk = c2;
+        my_base = C;
       }
       C += v;
     }
+    if (my_chunk != INT_MAX) atomicMin(&s_chunk, my_chunk);
   }
   __syncthreads();
+  // (rounding may let two neighbours claim: the first chunk wins, and only its
+  // claimant writes the base)
+  if (my_chunk == s_chunk) s_base = my_base;
   if (threadIdx.x == 0) {
     s_t = t;
-    s_base = -1.0;  // < 0 selects the "last positive element" rule
     if (s_chunk == INT_MAX) {  // rounding left t at or past the total
       int cs = 0;
       for (int c2 = nsr - 1; c2 >= 0; --c2)
@@ -1333,14 +1355,6 @@ __global__ void __launch_bounds__(NTH, 65536 / (NTH * kFinishMaxNreg)) k_finish(
       s_chunk = cs;
     }
     if (dbg_Z) dbg_Z[b] = Z / St;
-  }
-  __syncthreads();
-  // the owner of the chosen chunk publishes its exclusive prefix
-  if (s_chunk >= c0 && s_chunk < c1) {
-    double C = cexcl;
-    for (int c2 = c0; c2 < s_chunk; ++c2) C += __ldcg(&rp[c2].R);
-    const double v = __ldcg(&rp[s_chunk].R);
-    if (C <= t && t < C + v) s_base = C;
   }
   __syncthreads();
 
