@@ -1541,11 +1541,15 @@ __global__ void __launch_bounds__(NT) k_smc_resample(const double *__restrict__ 
 // row other than x_{i+1} are the candidates for the next-next token.  Order:
 // larger logit first, equal logits by ascending token id; a row with a NaN is
 // invalid.  One CTA per row:
-//   1. the thread maxima of the row give a lower bound tau of its k-th
-//      largest key (radix select on the top 16 key bits);
-//   2. a second pass (from L2) appends every non-excluded element with
-//      key >= tau to a shared buffer (about k of them for real logits) and
-//      checks for NaN;
+//   1. one pass over the row (HBM) keeps each thread's maximum, the maximum
+//      of each of its groups of vectors (top 16 key bits, in shared memory)
+//      and whether it met a NaN; the thread maxima give a lower bound tau of
+//      the row's k-th largest key (the largest 16-bit key bucket holding at
+//      least k of them, by bisection with block-wide counts);
+//   2. only the groups whose maximum reaches tau (about k of them for real
+//      logits) are read again (from L2), spread over all threads, and every
+//      non-excluded element with key >= tau goes to a shared buffer; when
+//      too many groups qualify (heavy ties) the whole row is read again;
 //   3. each candidate's rank (the number of candidates above it) places it;
 //      up to the buffer's size a bitonic sort of (key, ~index) does it
 //      instead, and when ties at the top overflow the buffer (e.g. a constant
@@ -1556,7 +1560,9 @@ __global__ void __launch_bounds__(NT) k_smc_resample(const double *__restrict__ 
 constexpr int kTopkThreads = 512;
 constexpr int kTopkCtasPerSm = 3;
 constexpr int kTopkMaxK = 256;
-constexpr int kTopkCap = 2048;  // candidate buffer (power of two)
+constexpr int kTopkCap = 2048;   // candidate buffer (power of two)
+constexpr int kTopkGroups = 16;  // vector groups per thread whose maxima pass 1 keeps
+constexpr int kTopkWork = 1024;  // qualifying groups pass 2 reads selectively, at most
 
 // order-preserving key: a larger logit has a larger key, -0 and +0 the same
 // key (equal logits); never 0 for a non-NaN value
@@ -1564,6 +1570,14 @@ __device__ __forceinline__ uint32_t logit_key(float f) {
   uint32_t u = __float_as_uint(f);
   if (u == 0x80000000u) u = 0u;
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// the logit of a key (logit_key is one-to-one but for -0 and +0, which share
+// a key: those are read back from the row)
+template <typename T>
+__device__ __forceinline__ float key_logit(uint32_t key, const T *p) {
+  if (key == 0x80000000u) return Dt<T>::load(p);
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
 }
 
 // f(index, logit) for every element of a row: scalar head, 16-byte vectors
@@ -1618,35 +1632,6 @@ __device__ __forceinline__ float vec_max_nan<float>(const uint4 &v) {
                    __uint_as_float(v.w), -INFINITY);
 }
 
-// The same walk as row_foreach, a whole 16-byte vector at a time:
-// fv(first element index, vector) for the body, fs(index, logit) for the
-// scalar head and tail.
-template <typename T, typename FV, typename FS>
-__device__ __forceinline__ void row_foreach_vec(const T *row, int V, FV fv, FS fs) {
-  constexpr int VEC = Dt<T>::VEC;
-  constexpr int UNR = 4;
-  const int head = row_head(row, (long long)V);
-  const int nvec = (V - head) / VEC;
-  if ((int)threadIdx.x < head) fs((int)threadIdx.x, Dt<T>::load(row + threadIdx.x));
-  const uint4 *pv = reinterpret_cast<const uint4 *>(row + head);
-  const int step = (int)blockDim.x;
-  for (int i0 = threadIdx.x; i0 < nvec; i0 += step * UNR) {
-    uint4 v[UNR];
-#pragma unroll
-    for (int u = 0; u < UNR; ++u) {
-      const int i = i0 + u * step;
-      v[u] = i < nvec ? __ldg(pv + i) : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int u = 0; u < UNR; ++u) {
-      const int i = i0 + u * step;
-      if (i < nvec) fv(head + i * VEC, v[u]);
-    }
-  }
-  const int t0 = head + nvec * VEC;
-  if (t0 + (int)threadIdx.x < V) fs(t0 + (int)threadIdx.x, Dt<T>::load(row + t0 + threadIdx.x));
-}
-
 // bitonic sort, descending, of n (a power of two, <= the block's reach) keys
 template <typename K>
 __device__ __forceinline__ void bitonic_desc(K *a, int n) {
@@ -1675,7 +1660,9 @@ __global__ void __launch_bounds__(kTopkThreads, kTopkCtasPerSm) k_topk_exclude(
     float *__restrict__ out_val) {
   __shared__ unsigned long long cand[kTopkCap];  // (key << 32) | ~index
   __shared__ unsigned hist[256];
-  __shared__ int s_n, s_bad, s_rem, s_cnt[kTopkThreads / 32];
+  __shared__ unsigned short s_gkey[kTopkGroups][kTopkThreads];  // group maxima (key >> 16)
+  __shared__ uint32_t s_work[kTopkWork];  // qualifying groups: thread | group << 16
+  __shared__ int s_n, s_bad, s_rem, s_nw, s_cnt[kTopkThreads / 32];
   __shared__ uint32_t s_prefix;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const long long r = blockIdx.x;
@@ -1689,27 +1676,35 @@ __global__ void __launch_bounds__(kTopkThreads, kTopkCtasPerSm) k_topk_exclude(
     s_n = 0;
     s_bad = 0;
   }
-  // 1. A lower bound tau of the row's k-th largest key: the thread maxima of
-  // the row are distinct elements, so their k-th largest is at most the
-  // row's.  It is found by a radix select on the top 16 key bits (two 8-bit
-  // histogram passes), and tau is the smallest key of its 16-bit bucket
-  // (exact for bf16 keys).  NaNs are left out here; the second pass finds
-  // them.
+  // 1. One pass over the row.  Thread t reads vectors t + 512*m in rounds of
+  // four (round j: m = 4j .. 4j+3); rounds are grouped ipg at a time into at
+  // most kTopkGroups groups whose maxima (top 16 bits of the key, 0 = no
+  // value) go to shared memory.  The thread maxima are distinct elements, so
+  // their k-th largest is at most the row's: tau is the smallest key of the
+  // largest 16-bit bucket holding at least k thread maxima (exact for bf16
+  // keys).  NaNs are left out of the maxima and mark the row invalid.
   constexpr int VEC = Dt<T>::VEC;
   const int head = row_head(row, (long long)V);
   const int nvec = (V - head) / VEC;
   const int P = nvec;
   const uint4 *pv = reinterpret_cast<const uint4 *>(row + head);
-  float mx = -INFINITY;
-  bool seen = false;
+  const int niter = (P + 4 * kTopkThreads - 1) / (4 * kTopkThreads);  // rounds
+  const int ipg = (niter + kTopkGroups - 1) / kTopkGroups;           // rounds per group
+  const int ngrp = ipg > 0 ? (niter + ipg - 1) / ipg : 0;
+  const int tail0 = head + nvec * VEC;
+  float mx = -INFINITY, gmx = -INFINITY;
+  bool seen = false, gseen = false, bad = false;
   auto take1 = [&](int v, float x) {
+    bad |= isnan(x);
     if (v != ex && !isnan(x)) {
       mx = fmaxf(mx, x);
       seen = true;
     }
   };
   if (tid < head) take1(tid, Dt<T>::load(row + tid));
-  for (int i0 = tid; i0 < P; i0 += 4 * kTopkThreads) {
+  if (tail0 + tid < V) take1(tail0 + tid, Dt<T>::load(row + tail0 + tid));
+  for (int j = 0; j < niter; ++j) {
+    const int i0 = tid + j * 4 * kTopkThreads;
     uint4 w[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -1726,62 +1721,49 @@ __global__ void __launch_bounds__(kTopkThreads, kTopkCtasPerSm) k_topk_exclude(
         float x[VEC];
         Dt<T>::unpack(w[u], x);
 #pragma unroll
-        for (int e2 = 0; e2 < VEC; ++e2) take1(v0 + e2, x[e2]);
+        for (int e2 = 0; e2 < VEC; ++e2) {
+          bad |= isnan(x[e2]);
+          if (v0 + e2 != ex && !isnan(x[e2])) {
+            gmx = fmaxf(gmx, x[e2]);
+            gseen = true;
+          }
+        }
       } else {
-        mx = fmaxf(mx, m);
+        gmx = fmaxf(gmx, m);
+        gseen = true;
+      }
+    }
+    if ((j + 1) % ipg == 0 || j + 1 == niter) {  // the group ends
+      s_gkey[j / ipg][tid] = gseen ? (unsigned short)(logit_key(gmx) >> 16) : (unsigned short)0;
+      if (gseen) {
+        mx = fmaxf(mx, gmx);
         seen = true;
       }
+      gmx = -INFINITY;
+      gseen = false;
     }
   }
   const uint32_t tkey = seen ? logit_key(mx) : 0u;  // 0: no value (below every key)
-  uint32_t prefix = 0;
-  int rem = k;
-  for (int shift = 24; shift >= 16; shift -= 8) {
-    for (int i = tid; i < 256; i += kTopkThreads) hist[i] = 0;
-    __syncthreads();
-    if (shift == 24 || (tkey >> 24) == (prefix >> 24)) atomicAdd(&hist[(tkey >> shift) & 255u], 1u);
-    __syncthreads();
-    if (warp == 0) {
-      // lane l holds buckets 255 - 8l - j, j < 8 (from the top); find the
-      // bucket where the count from the top reaches rem
-      unsigned c8 = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) c8 += hist[255 - 8 * lane - j];
-      unsigned incl = c8;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const unsigned y = __shfl_up_sync(FULL, incl, o);
-        if (lane >= o) incl += y;
-      }
-      const unsigned excl = incl - c8;
-      const bool here = excl < (unsigned)rem && incl >= (unsigned)rem;
-      const unsigned who = __ballot_sync(FULL, here);
-      if (who != 0u && lane == __ffs(who) - 1) {
-        unsigned cum = excl;
-        int d = 255 - 8 * lane;
-        for (int j = 0; j < 8; ++j, --d) {
-          if (cum + hist[d] >= (unsigned)rem) break;
-          cum += hist[d];
-        }
-        s_rem = rem - (int)cum;
-        s_prefix = prefix | ((uint32_t)d << shift);
-      } else if (who == 0u && lane == 0) {  // fewer than rem keys in all: every key qualifies
-        s_rem = rem;
-        s_prefix = prefix;
-      }
-    }
-    __syncthreads();
-    prefix = s_prefix;
-    rem = s_rem;
-    __syncthreads();
+  // bisection over the 16-bit buckets with block-wide counts
+  uint32_t blo = 0, bhi = 65535;
+  while (blo < bhi) {
+    const uint32_t mid = (blo + bhi + 1) >> 1;
+    if (__syncthreads_count(tkey >= (mid << 16)) >= k) blo = mid;
+    else bhi = mid - 1;
   }
-  const uint32_t tau = prefix;  // the bucket's smallest key (low 16 bits 0)
-  // 2. A second pass over the row (now in L2): every non-excluded key >= tau
-  // goes to the candidate buffer (a vector is unpacked only when its max
-  // reaches tau or is NaN); a NaN anywhere makes the row invalid.
-  bool bad = false;
+  const uint32_t tau = blo << 16;  // the bucket's smallest key (low 16 bits 0)
+  // 2. The qualifying groups (maximum >= tau) go to a work list; every thread
+  // then takes vectors of the listed groups in turn (one L2 round trip for
+  // about k groups), and every non-excluded key >= tau goes to the candidate
+  // buffer (a vector is unpacked only when its max reaches tau).
+  if (tid == 0) s_nw = 0;
+  __syncthreads();
+  for (int gi = 0; gi < ngrp; ++gi)
+    if ((uint32_t)s_gkey[gi][tid] << 16 >= tau && s_gkey[gi][tid] != 0) {
+      const int pos = atomicAdd(&s_nw, 1);
+      if (pos < kTopkWork) s_work[pos] = (uint32_t)tid | ((uint32_t)gi << 16);
+    }
   auto scalar2 = [&](int v, float x) {
-    bad |= isnan(x);
     const uint32_t key = logit_key(x);
     if (v != ex && key >= tau && !isnan(x)) {
       const int pos = atomicAdd(&s_n, 1);
@@ -1789,15 +1771,57 @@ __global__ void __launch_bounds__(kTopkThreads, kTopkCtasPerSm) k_topk_exclude(
         cand[pos] = ((unsigned long long)key << 32) | (unsigned)(0xFFFFFFFFu - (unsigned)v);
     }
   };
-  row_foreach_vec(row, V, [&](int v0, const uint4 &w) {
+  auto vec2 = [&](int i, const uint4 &w) {
     const float m = vec_max_nan<T>(w);
-    if (isnan(m) || logit_key(m) >= tau) {
+    if (!isnan(m) && logit_key(m) >= tau) {
       float x[VEC];
       Dt<T>::unpack(w, x);
+      const int v0 = head + i * VEC;
 #pragma unroll
       for (int e2 = 0; e2 < VEC; ++e2) scalar2(v0 + e2, x[e2]);
     }
-  }, scalar2);
+  };
+  __syncthreads();
+  const int nw = s_nw;
+  if (tid < head) scalar2(tid, Dt<T>::load(row + tid));
+  if (tail0 + tid < V) scalar2(tail0 + tid, Dt<T>::load(row + tail0 + tid));
+  if (nw <= kTopkWork) {
+    const int per = 4 * ipg;  // vectors of one group
+    for (int f0 = tid; f0 < nw * per; f0 += 4 * kTopkThreads) {
+      uint4 w[4];
+      int iv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int f = f0 + u * kTopkThreads;
+        iv[u] = -1;
+        if (f < nw * per) {
+          const uint32_t e = s_work[f / per];
+          const int r2 = f % per;
+          const int j = (int)(e >> 16) * ipg + r2 / 4;
+          const int i = (int)(e & 0xFFFFu) + (4 * j + (r2 & 3)) * kTopkThreads;
+          if (j < niter && i < P) iv[u] = i;
+        }
+        w[u] = iv[u] >= 0 ? __ldg(pv + iv[u]) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (iv[u] >= 0) vec2(iv[u], w[u]);
+    }
+  } else {  // many groups reach tau (heavy ties): the whole row again
+    for (int i0 = tid; i0 < P; i0 += 4 * kTopkThreads) {
+      uint4 w[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * kTopkThreads;
+        w[u] = i < P ? __ldg(pv + i) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * kTopkThreads;
+        if (i < P) vec2(i, w[u]);
+      }
+    }
+  }
   if (__any_sync(FULL, bad) && lane == 0) s_bad = 1;
   __syncthreads();
   if (s_bad) {  // invalid row
@@ -1820,7 +1844,7 @@ __global__ void __launch_bounds__(kTopkThreads, kTopkCtasPerSm) k_topk_exclude(
       if (rank < k) {
         const int v = (int)(0xFFFFFFFFu - (unsigned)(c & 0xFFFFFFFFull));
         oi[rank] = v;
-        if (ov) ov[rank] = Dt<T>::load(row + v);
+        if (ov) ov[rank] = key_logit((uint32_t)(c >> 32), row + v);
       }
     }
     for (int i = n + tid; i < k; i += blockDim.x) {

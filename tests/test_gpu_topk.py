@@ -5,7 +5,8 @@ rows (k = 60, the LogitSpec page's figure, excluding the draft tokens), fp32
 rows of 151936, k = 1 and 256, quantised logits with many ties (the fast
 path), constant rows (ties overflow the candidate buffer: the radix-select
 path), -inf entries, rows shorter than k, odd V with misaligned rows, rows
-picked by index, NaN rows, bad arguments."""
+picked by index, NaN rows (also a NaN among values far below the top k
+of a long row), exclusions at vector-group edges, bad arguments."""
 import numpy as np
 import pytest
 
@@ -96,3 +97,28 @@ def test_nan_rows_and_bad_arguments():
     for k, stride in ((0, 8), (257, 8), (4, 7)):
         assert sd.specdec_topk_exclude(p, stride, None, 2, 8, sd.SPECDEC_F32, None, k, p, p, s) \
             == sd.SPECDEC_EINVAL
+
+
+def test_long_rows_nan_outside_the_top_groups_then_clean_call():
+    """Long rows (fp32, 12500 vectors: 7 rounds of 4 vectors per thread, one
+    vector group per round): a NaN among values far below the top k and one
+    in the last element make those rows invalid (the first pass, which reads
+    every element, finds them); exclusions sit on round edges.  A following
+    clean call must be exact."""
+    rng = np.random.default_rng(11)
+    V = 50000
+    rows = rng.normal(0, 3, (4, V)).astype(np.float32)
+    rows[1, 24992:25008] = -50.0
+    rows[1, 25000] = np.nan
+    rows[2, V - 1] = np.nan
+    seg = 4 * 512 * 4          # elements of one round of the 512 threads
+    ex = np.array([seg, 2 * seg - 1, 0, V - 1])
+    sd.specdec_device_errors(None)
+    _check(rows, "f32", 60, ex)
+    st, flags = sd.specdec_device_errors(None)
+    assert flags & sd.SPECDEC_ERR_LOGITS
+    clean = rng.normal(0, 3, (2, V)).astype(np.float32)
+    _check(clean, "f32", 60, np.array([seg * 4 * 3, 5]))
+    st, flags = sd.specdec_device_errors(None)
+    assert not (flags & sd.SPECDEC_ERR_LOGITS)
+    _check(inputs.f32_to_bf16_bits(rows[[0, 3]]), "bf16", 256, ex[[0, 3]])
