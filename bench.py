@@ -59,6 +59,9 @@ def parse():
     ap.add_argument("--chained", choices=["on", "off"], default="on",
                     help="also time specdec_verify_chained (an intermediate tensor of the "
                          "target's shape, the target logits as the final layer)")
+    ap.add_argument("--early-exit-large", choices=["on", "off"], default="on",
+                    help="also time the full call and early exit on the large fp32 workload's "
+                         "shape (K=8, V=151936) at 64 sequences per rank")
     ap.add_argument("--topk", choices=["on", "off"], default="on",
                     help="also time specdec_topk_exclude (k=60) over the target's draft rows")
     ap.add_argument("--smc", choices=["on", "off"], default="on",
@@ -441,6 +444,63 @@ def run_cuda(args):
                    note="the bench shape with draft noise 1.5 for every sequence")
         early["low_acceptance"] = low
         del lb, lcalls
+
+        # a workload where the rows early exit leaves unread outweigh its second
+        # finish chain: the large fp32 workload's shape (K = 8, V = 151936) at
+        # 64 sequences per rank, at its own draft noise and at 1.5
+        if args.early_exit_large == "on":
+            big = {}
+            LB = 64
+            for tag, sig in (("default_noise", None), ("noise_1.5", 1.5)):
+                xb = sdist.generate_shard("large_b256_k8_v151936_f32", rank, world, per_rank=LB,
+                                          sigma=sig)
+                wb = inputs.WORKLOADS["large_b256_k8_v151936_f32"]
+                tvb = tview if wb.dtype == w.dtype else (
+                    (lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16))
+                    if wb.dtype == "bf16" else (lambda a: torch.from_numpy(a)))
+                dtb = sd.SPECDEC_BF16 if wb.dtype == "bf16" else sd.SPECDEC_F32
+                bb = [dict(t=tvb(xb.target).to(dev), d=tvb(xb.draft).to(dev),
+                           tok=torch.from_numpy(xb.tokens).to(dev),
+                           ua=torch.from_numpy(xb.u_accept).to(dev),
+                           ur=torch.from_numpy(xb.u_resample).to(dev),
+                           T=torch.from_numpy(xb.temperature).to(dev),
+                           ot=torch.empty((LB, xb.K + 1), dtype=torch.int32, device=dev),
+                           on=torch.empty((LB,), dtype=torch.int32, device=dev)) for _ in range(2)]
+                bc = [(b["t"].data_ptr(), b["d"].data_ptr(), b["tok"].data_ptr(), b["ua"].data_ptr(),
+                       b["ur"].data_ptr(), b["T"].data_ptr(), LB, xb.K, xb.V, dtb,
+                       b["ot"].data_ptr(), b["on"].data_ptr(), sp) for b in bb]
+                leg = {}
+                for key, f in (("full_ms_per_step", fn), ("early_exit_ms_per_step", fe)):
+                    for i in range(3):
+                        if f(*bc[i % 2]) != 0:
+                            raise RuntimeError("verify failed on the large-shape batch")
+                    torch.cuda.synchronize()
+                    barrier()
+                    torch.cuda.synchronize()
+                    h0 = torch.cuda.Event(enable_timing=True)
+                    h1 = torch.cuda.Event(enable_timing=True)
+                    h0.record(stream)
+                    for i in range(args.steps):
+                        f(*bc[i % 2])
+                    h1.record(stream)
+                    torch.cuda.synchronize()
+                    barrier()
+                    leg[key] = sdist.max_over_ranks(h0.elapsed_time(h1), dev) / args.steps
+                    if key == "full_ms_per_step":
+                        big_tok = bb[0]["ot"].cpu().numpy().copy()
+                Pb = 2 if xb.K >= 2 else xb.K
+                n_b = bb[0]["on"].cpu().numpy()
+                rows_b = int(np.sum(np.where(n_b >= Pb, 2 * xb.K + 1, 2 * Pb)))
+                leg.update(rows_read_fraction=rows_b / (LB * (2 * xb.K + 1)),
+                           mean_accepted=float(np.mean(n_b)),
+                           tokens_equal_full_call=bool(np.array_equal(bb[0]["ot"].cpu().numpy(),
+                                                                       big_tok)))
+                big[tag] = leg
+                del bb, bc, xb
+                torch.cuda.empty_cache()
+            early["large_fp32_shape"] = dict(
+                big, workload="large_b256_k8_v151936_f32 recipe, B=%d per rank" % LB,
+                bytes_per_step=LB * world * 17 * 151936 * 4)
 
     # ---- SMC-SD weight step on the same logits (groups of 8 particles) -------
     smc_line = None
