@@ -668,8 +668,8 @@ def run_cuda(args):
         "gpu_launches": launches,
     }
     if kern:
-        # one verify step launches the sweep once per wave of sequences; the
-        # achieved rate is the algorithmic bytes of a launch over its mean time
+        # launches of the sweep per step (one for the full call); the achieved
+        # rate is the algorithmic bytes of a launch over its mean time
         st_ms, st_n = kern["k_row_stats"]
         per_launch = floor * args.steps / max(st_n, 1)
         avg = st_ms / max(st_n, 1)

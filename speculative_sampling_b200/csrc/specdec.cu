@@ -184,8 +184,9 @@ __device__ __forceinline__ float half_max_nan(float v) {
 // ---------------------------------------------------------------------------
 // kernel 1: softmax statistics of every row
 // ---------------------------------------------------------------------------
-// A sweep reads the rows of a range of sequences (a wave of the batch), in
-// sequence order, cut into tiles of CW*32*U 16-byte vectors (16 KB for U = 4);
+// A sweep reads the rows of its window (every row of the batch, or some
+// positions of it), in sequence order, cut into tiles of CW*32*U 16-byte
+// vectors (16 KB for U = 4);
 // CTA g of a grid of G owns the contiguous tile range [g*T/G, (g+1)*T/G).
 //
 // Warp specialisation: one producer warp streams tiles with cp.async.bulk
