@@ -345,10 +345,6 @@ __device__ __forceinline__ float2 exp2_fma2(float2 a) {
   return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
                      __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
-// 1: the sweep's exponent arguments with log2(e)/T as one fp32 value
-#ifndef SPECDEC_SINGLE_SCALE
-#define SPECDEC_SINGLE_SCALE 0
-#endif
 // pairs of each 16-byte vector whose exponentials the sweep takes on the FMA
 // pipe (the rest on MUFU)
 #ifndef SPECDEC_EXP_FMA_PAIRS
@@ -426,11 +422,7 @@ __device__ __forceinline__ void vec_fold(const uint4 &v, RunStat &q, Scale c, fl
 #pragma unroll
   for (int k = 0; k < N; ++k) {
     const float2 d = __fadd2_rn(x[k], nr);
-#if SPECDEC_SINGLE_SCALE
-    const float2 a = __fmul2_rn(d, __fadd2_rn(hi, lo));
-#else
     const float2 a = __ffma2_rn(d, hi, __fmul2_rn(d, lo));
-#endif
     if (k < SPECDEC_EXP_FMA_PAIRS)
       e[k] = exp2_fma2(a);
     else
