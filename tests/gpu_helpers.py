@@ -14,6 +14,12 @@ import speculative_sampling_b200 as sd
 # error of a normaliser is a few 1e-7 relative; 1e-5 leaves a wide margin while
 # still catching any dropped term or wrong scale.
 RTOL = 1e-5
+# Z (the residual mass, in probability units) is a difference of probabilities:
+# sum max(0, p - q).  p and q carry the relative error of their normalisers
+# (~1.6e-7 measured), so Z's absolute error is up to ~3e-7 however small Z is;
+# when p and q nearly agree (Z of a few 1e-6, met by the fuzzed shapes) that is
+# several percent of Z.  Z is compared within RTOL relative plus Z_ATOL.
+Z_ATOL = 1e-6
 # Decisions whose oracle margin is below this band may legitimately differ.
 BAND = 1e-6
 # Canary bands: every device output of the parity tests sits between two bands
@@ -193,8 +199,9 @@ def compare(g: dict, o: dict, seqs=None, rtol=RTOL, band=BAND, stats=True,
     e_q = rel(g["q_x"][reach], o["q_x"][reach])
     assert e_p.max(initial=0) <= rtol, ("p(x)", e_p.max())
     assert e_q.max(initial=0) <= rtol, ("q(x)", e_q.max())
-    e_z = rel(g["Z"][same], o["Z"][same])
-    assert e_z.max(initial=0) <= rtol, ("Z", e_z.max())
+    zg, zo = g["Z"][same], o["Z"][same]
+    e_z = rel(zg, zo)
+    assert np.all(np.abs(zg - zo) <= rtol * np.abs(zo) + Z_ATOL), ("Z", e_z.max(initial=0))
     res.update(max_rel_row_sum=float(e_s.max(initial=0)), max_rel_px=float(e_p.max(initial=0)),
                max_rel_qx=float(e_q.max(initial=0)), max_rel_Z=float(e_z.max(initial=0)))
     return res

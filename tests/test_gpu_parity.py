@@ -159,3 +159,34 @@ def test_empty_batch():
                        e((0,), dtype=torch.float32, device="cuda"),
                        e((0,), dtype=torch.float32, device="cuda"))
     assert ot.shape == (0, 6) and on.shape == (0,)
+
+
+def _fuzz_cases(n=24, seed=2026):
+    """Seeded random shapes over the four recipes: B in [1, 48], K in [1, 12],
+    V log-uniform in [1, 70000] (odd and even, so rows take every alignment),
+    per-sequence temperatures in [0.2, 4]."""
+    rng = np.random.default_rng(seed)
+    names = ["tiny_b1_k4_v1000_f32", "batched_b64_k5_v128256_bf16", "mix_b128_k4_v32000_bf16",
+             "large_b256_k8_v151936_f32"]
+    cases = []
+    for i in range(n):
+        name = names[i % len(names)]
+        B = int(rng.integers(1, 49))
+        K = int(rng.integers(1, 13))
+        V = int(np.exp(rng.uniform(0.0, np.log(70000.0))))
+        T = np.exp(rng.uniform(np.log(0.2), np.log(4.0), B)).astype(np.float32)
+        cases.append((i, name, B, K, max(V, 1), T))
+    return cases
+
+
+@pytest.mark.parametrize("case", _fuzz_cases(), ids=lambda c: "fuzz%02d_%s_B%d_K%d_V%d" % c[:5])
+def test_parity_fuzzed_shapes(case):
+    """The full call and early exit against the oracle on seeded random shapes:
+    every sequence without a boundary draw bit-exact, statistics within the
+    tolerance, canaries intact (gpu_helpers)."""
+    _, name, B, K, V, T = case
+    x = inputs.generate(name, B=B, K=K, V=V)
+    x.temperature[:] = T
+    o = H.oracle_verify(x)
+    H.compare(H.gpu_verify(x), o)
+    H.compare(H.gpu_verify(x, debug=False, early_exit=True), o, stats=False)
