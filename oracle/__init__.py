@@ -110,5 +110,14 @@ def verify(*args, **kw) -> dict:
 def boundary_mask(res: dict, band: float = 1e-6) -> np.ndarray:
     """Sequences whose acceptance or sampling decision lies within ``band`` of a
     threshold (the decisions a correct lower-precision implementation may take
-    either way)."""
-    return (res["margin_accept"] < band) | (res["margin_sample"] < band)
+    either way).
+
+    Acceptance: |u - p/q| < band.  Token draw: the distance from u*Z to the
+    nearer edge of the chosen cell of the cumulative sum, in probability units
+    (margin_sample is that distance divided by Z, so it is multiplied back):
+    the residual max(0, p - q) is a difference of probabilities, which any
+    implementation whose normalisers carry a relative error of order 1e-7 knows
+    only to that absolute precision, however small Z is.  For the bonus row
+    Z = 1 and both readings agree."""
+    draw = np.asarray(res["margin_sample"]) * np.where(np.isfinite(res["Z"]), res["Z"], 1.0)
+    return (res["margin_accept"] < band) | (draw < band)

@@ -104,7 +104,8 @@ def verify_chained(final, inter, draft, tokens, u_accept1, u_resample1, u_accept
             C = np.cumsum(r)
             t = ur2[b] * C[-1]
             lo = C[y - 1] if y > 0 else 0.0
-            margin[b] = min(margin[b], min(abs(t - lo), abs(C[y] - t)) / C[-1])
+            # (in probability units: see oracle.boundary_mask)
+            margin[b] = min(margin[b], min(abs(t - lo), abs(C[y] - t)))
             emitted[b] = n2 + 1
         else:
             emitted[b] = m

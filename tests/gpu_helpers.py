@@ -176,7 +176,8 @@ def compare(g: dict, o: dict, seqs=None, rtol=RTOL, band=BAND, stats=True,
     # boundary sequences over valid ones, and the count of their boundary draws
     # (an acceptance test or the token draw within `band` of its threshold)
     nb_acc = int(np.sum(valid & (o["margin_accept"] < band)))
-    nb_smp = int(np.sum(valid & (o["margin_sample"] < band)))
+    nb_smp = int(np.sum(valid & (o["margin_sample"] * np.where(np.isfinite(o["Z"]), o["Z"], 1.0)
+                                 < band)))
     res = {"sequences": int(on.size), "valid": int(valid.sum()), "boundary": int(bnd.sum()),
            "draws": draws, "mismatched": int(differ.sum()),
            "boundary_rate": float(bnd.sum()) / max(int(valid.sum()), 1),
