@@ -109,3 +109,30 @@ def test_smc_step_rejects_bad_arguments():
                                p, p, p, None, s) == sd.SPECDEC_EINVAL
     assert sd.specdec_smc_step(p, p, p, p, p, None, p, -1.0, 4, 4, 2, 8, sd.SPECDEC_F32, p, p, p,
                                p, None, s) == sd.SPECDEC_EINVAL
+
+
+def _smc_fuzz(n=12, seed=99):
+    rng = np.random.default_rng(seed)
+    names = ["tiny_b1_k4_v1000_f32", "batched_b64_k5_v128256_bf16", "mix_b128_k4_v32000_bf16",
+             "large_b256_k8_v151936_f32"]
+    out = []
+    for i in range(n):
+        N = int(rng.choice([1, 2, 3, 4, 8, 16]))
+        G = int(rng.integers(1, 9))
+        K = int(rng.integers(1, 13))
+        V = max(1, int(np.exp(rng.uniform(0.0, np.log(40000.0)))))
+        thr = float(rng.choice([0.0, 0.3, 0.7, 1.0]))
+        T = np.exp(rng.uniform(np.log(0.2), np.log(4.0), N * G)).astype(np.float32)
+        lw = rng.normal(0, 1.5, N * G) if i % 2 else None
+        out.append((i, names[i % 4], N, G, K, V, thr, T, lw))
+    return out
+
+
+@pytest.mark.parametrize("case", _smc_fuzz(), ids=lambda c: "sfuzz%02d_%s_N%d_G%d_K%d_V%d" % c[:6])
+def test_smc_step_fuzzed_shapes(case):
+    """Seeded random group sizes, shapes, thresholds, temperatures and
+    incoming log-weights against the oracle."""
+    i, name, N, G, K, V, thr, T, lw = case
+    x = inputs.generate(name, B=N * G, K=K, V=V)
+    x.temperature[:] = T
+    _check(x, N, thr, lw, _uniforms(G, 100 + i))
