@@ -190,3 +190,13 @@ def test_parity_fuzzed_shapes(case):
     o = H.oracle_verify(x)
     H.compare(H.gpu_verify(x), o)
     H.compare(H.gpu_verify(x, debug=False, early_exit=True), o, stats=False)
+
+
+def test_parity_many_sequences():
+    """B = 2048 (the finish grid takes several waves of CTAs, one CTA per
+    sequence; each sweep CTA holds many rows), every sequence against the
+    oracle, for the full call and early exit."""
+    x = inputs.generate("mix_b128_k4_v32000_bf16", B=2048, V=16000)
+    o = H.oracle_verify(x)
+    print("B=2048", H.compare(H.gpu_verify(x), o))
+    H.compare(H.gpu_verify(x, debug=False, early_exit=True), o, stats=False)
