@@ -328,8 +328,7 @@ const char *specdec_error_string(specdec_status s);
  *     0.4 MiB and fits up to B=837; K=8,V=151936 fp32 needs 2.3 MiB at B=256
  *     and fits up to B=449).
  *   - The first call on a device looks up the array's device address (once
- *     per device, with that device current); make that first call before any
- *     stream capture on that device.
+ *     per device, with that device current).
  *   - All calls share the one array, which keeps the last call's contents:
  *     calls whose executions overlap on the GPU (on different streams, or
  *     from different host threads) race on it and must be serialised by the
