@@ -40,6 +40,18 @@ METRIC = "verify GB/s (% of HBM peak) and rows/s at B=64 K=5 V=128256 bf16"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 2 ** 20
+# Device cycles of a delay queued on the stream just before a timed region's
+# start event (about 0.3 ms at 2 GHz): while the device waits, the host queues
+# the region's first launches, so the events bracket the device's time for the
+# K steps and not the host's issue of the first one.  Nothing of the verify
+# runs during the delay, which lies outside the region.
+QUEUE_DELAY_CYCLES = 600_000
+
+
+def start_region(torch, ev, stream):
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(QUEUE_DELAY_CYCLES)
+    ev.record(stream)
 
 
 def parse():
@@ -327,7 +339,7 @@ def run_cuda(args):
     e1 = torch.cuda.Event(enable_timing=True)
     sampler.go_fast()
     tw0 = time.perf_counter()
-    e0.record(stream)
+    start_region(torch, e0, stream)
     for i in range(args.steps):
         step(i)
     e1.record(stream)
@@ -386,7 +398,7 @@ def run_cuda(args):
         torch.cuda.synchronize()
         f0 = torch.cuda.Event(enable_timing=True)
         f1 = torch.cuda.Event(enable_timing=True)
-        f0.record(stream)
+        start_region(torch, f0, stream)
         for i in range(args.steps):
             fe(*calls[i % ncopies])
         f1.record(stream)
@@ -427,7 +439,7 @@ def run_cuda(args):
             torch.cuda.synchronize()
             g0 = torch.cuda.Event(enable_timing=True)
             g1 = torch.cuda.Event(enable_timing=True)
-            g0.record(stream)
+            start_region(torch, g0, stream)
             for i in range(args.steps):
                 f(*lcalls[i % ncopies])
             g1.record(stream)
@@ -479,7 +491,7 @@ def run_cuda(args):
                     torch.cuda.synchronize()
                     h0 = torch.cuda.Event(enable_timing=True)
                     h1 = torch.cuda.Event(enable_timing=True)
-                    h0.record(stream)
+                    start_region(torch, h0, stream)
                     for i in range(args.steps):
                         f(*bc[i % 2])
                     h1.record(stream)
@@ -527,7 +539,7 @@ def run_cuda(args):
         torch.cuda.synchronize()
         s0 = torch.cuda.Event(enable_timing=True)
         s1 = torch.cuda.Event(enable_timing=True)
-        s0.record(stream)
+        start_region(torch, s0, stream)
         for i in range(args.steps):
             smc(i)
         s1.record(stream)
@@ -564,7 +576,7 @@ def run_cuda(args):
         torch.cuda.synchronize()
         c0 = torch.cuda.Event(enable_timing=True)
         c1 = torch.cuda.Event(enable_timing=True)
-        c0.record(stream)
+        start_region(torch, c0, stream)
         for i in range(args.steps):
             ch(i)
         c1.record(stream)
@@ -603,7 +615,7 @@ def run_cuda(args):
         torch.cuda.synchronize()
         k0 = torch.cuda.Event(enable_timing=True)
         k1 = torch.cuda.Event(enable_timing=True)
-        k0.record(stream)
+        start_region(torch, k0, stream)
         for i in range(args.steps):
             tk(i)
         k1.record(stream)
@@ -661,6 +673,8 @@ def run_cuda(args):
                    "B_total": B * world, "parallelism": f"dp{world}",
                    "l2": f"inputs rotate over {ncopies} device copies "
                          f"({ncopies * floor / 1e6:.0f} MB) > 126 MB L2"},
+        "timing": "CUDA events around the K steps on their stream; a device delay queued "
+                  "before the start event lets the host queue the first launches",
         "rows_per_s": rows / (ms_step * 1e-3),
         "sequences_per_s": B * world / (ms_step * 1e-3),
         "pct_of_hbm_peak": {f"of_{peak_kind}_{peak:.0f}GBs": 100.0 * gbs / world / peak,
