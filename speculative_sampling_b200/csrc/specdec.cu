@@ -222,6 +222,11 @@ constexpr int NSTAGE = 3;           // depth of the shared-memory ring
 constexpr unsigned long long kWaitNs = 2000000000ull;  // a wait gives up after 2 s by default
 constexpr unsigned kSuspendNs = 20000;  // longest sleep of one try_wait round
 constexpr int kStatsCtasPerSm = SPECDEC_SWEEP_CTAS_PER_SM;  // sweep CTAs per SM the grid is sized for
+// tiles at the start of each sweep CTA's range prefetched into L2 before the
+// CTA waits for the previous kernel on the stream
+#ifndef SPECDEC_SWEEP_PREFETCH_TILES
+#define SPECDEC_SWEEP_PREFETCH_TILES 1
+#endif
 constexpr int kFinishUW = 4;        // vectors per lane in a k_finish chunk
 constexpr int kFinishThreads = 256;   // threads of a k_finish CTA
 constexpr int kFinishCtasPerSm = 4;   // k_finish grids fit one wave of this many CTAs per SM
@@ -283,6 +288,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, unsigned parity,
 // part of it)
 __device__ __forceinline__ void consumer_sync() {
   asm volatile("bar.sync 1, %0;" ::"r"(NTC) : "memory");
+}
+// hint: bring a global range into L2 (16-byte aligned address, size a
+// multiple of 16); reads nothing into the SM and completes on its own
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, unsigned bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 // global -> shared bulk copy completing on an mbarrier (16-byte aligned
 // addresses, size a multiple of 16)
@@ -563,6 +573,27 @@ __global__ void SPECDEC_SWEEP_BOUNDS k_row_stats(const T *__restrict__ target,
     }
     s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  // Before waiting for the previous kernel: the first tiles of this CTA's
+  // range are requested into L2.  A prefetch reads nothing into the CTA, and
+  // L2 is coherent, so whatever that kernel still writes is what the copies
+  // below see; when it is the previous call's finish pass, these bytes stream
+  // while its draw runs.  (A sweep over the open sequences only reads a state
+  // written by the previous kernel and prefetches nothing.)
+  if (SPECDEC_SWEEP_PREFETCH_TILES > 0 && warp == CW && lane == 0 && g.state == nullptr &&
+      t0 < t1) {
+    RowCursor<T> pc;
+    pc.start(target, draft, g, t0);
+    long long t = t0;
+    const long long tend = t0 + SPECDEC_SWEEP_PREFETCH_TILES < t1 ? t0 + SPECDEC_SWEEP_PREFETCH_TILES : t1;
+    while (t < tend) {
+      const long long row = t / g.tpr;
+      if (row != pc.row) pc.next_row(target, draft, g);
+      const long long v0 = (t - row * g.tpr) * TV;
+      const long long v1 = (v0 + TV < pc.nvec) ? v0 + TV : pc.nvec;
+      if (v1 > v0) bulk_prefetch_l2(pc.pv + v0, (unsigned)(v1 - v0) * 16u);
+      ++t;
+    }
   }
   __syncthreads();
   cudaGridDependencySynchronize();
