@@ -24,9 +24,10 @@
 //                   resampling per group of particles.
 //   k_topk_exclude  top-k token ids of a row leaving one token out.
 // Kernels are launched with programmatic dependent launch: each signals its
-// dependents at its start and waits for its predecessor
+// dependents early and waits for its predecessor
 // (cudaGridDependencySynchronize) only where it first needs its results; the
-// call's first kernel waits before it reads anything.
+// call's first kernel waits before it reads anything (the statistics sweep
+// only requests its first tiles into L2 before that).
 //
 // Arithmetic: logits are widened exactly to fp32.  Exponentials are
 // 2^((z - m) * c) with c = log2(e)/T carried as an fp32 pair (hi + lo, with
@@ -1690,6 +1691,11 @@ __global__ void __launch_bounds__(kTopkThreads, kTopkCtasPerSm) k_topk_exclude(
   __shared__ uint32_t s_prefix;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const long long r = blockIdx.x;
+  // Programmatic dependent launch: this CTA may be placed while the previous
+  // kernel on the stream drains; it reads every input after waiting for it,
+  // and lets the next kernel be placed as this grid drains.
+  cudaGridDependencySynchronize();
+  cudaTriggerProgrammaticLaunchCompletion();
   const long long src = row_index ? row_index[r] : r;
   const T *row = logits + src * row_stride;
   const int ex0 = exclude ? exclude[r] : -1;
@@ -2611,15 +2617,16 @@ specdec_status specdec_topk_exclude(const void *logits, long long row_stride,
     return SPECDEC_EINVAL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   LaunchTimer lt(KID_TOPK, st);
+  cudaError_t e;
   if (dtype == SPECDEC_BF16)
-    k_topk_exclude<__nv_bfloat16><<<(unsigned)rows, kTopkThreads, 0, st>>>(
-        static_cast<const __nv_bfloat16 *>(logits), row_stride, row_index, V, exclude, k, out_idx,
-        out_val);
+    e = launch_pdl(k_topk_exclude<__nv_bfloat16>, (unsigned)rows, kTopkThreads, 0, st,
+                   static_cast<const __nv_bfloat16 *>(logits), row_stride, row_index, V, exclude,
+                   k, out_idx, out_val);
   else
-    k_topk_exclude<float><<<(unsigned)rows, kTopkThreads, 0, st>>>(
-        static_cast<const float *>(logits), row_stride, row_index, V, exclude, k, out_idx,
-        out_val);
-  return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ECUDA;
+    e = launch_pdl(k_topk_exclude<float>, (unsigned)rows, kTopkThreads, 0, st,
+                   static_cast<const float *>(logits), row_stride, row_index, V, exclude, k,
+                   out_idx, out_val);
+  return e == cudaSuccess ? SPECDEC_OK : SPECDEC_ECUDA;
 }
 
 specdec_status specdec_verify_chained_ex(
