@@ -477,6 +477,7 @@ struct StatsGeom {
   int pcw;          // partials per (row, CTA): CW (one per consumer warp, no CTA
                     // barrier) or 1 (the warps' partials combined per CTA, for rows
                     // shared by many CTAs, so that the finish pass reads fewer)
+  int late_sync;    // (instantiations with LATE only) see k_row_stats
 };
 __device__ __forceinline__ bool seq_active(const StatsGeom &g, long long b) {
   return g.state == nullptr || __ldcg(g.state + b) == kSeqActive;
@@ -548,7 +549,14 @@ struct RowCursor {
 // (cudaGridDependencySynchronize) after the shared-memory setup, before it
 // reads an input or touches the workspace, and only then lets the dependent
 // finish pass launch.
-template <typename T, int U>
+// With LATE and g.late_sync set: the previous kernel on the stream writes
+// nothing this sweep reads or writes but the finish pass's tickets (a later
+// stage of the same call): stream at once, and let one thread wait for that
+// kernel (then zero the tickets) at the end, so that this grid still
+// completes after it.  (Both sweeps of a call that has such a stage use the
+// LATE instantiation: the second stage's CTAs were measured to overlap the
+// first stage's finish only when they run the same kernel as its sweep.)
+template <typename T, int U, bool LATE = false>
 __global__ void SPECDEC_SWEEP_BOUNDS k_row_stats(const T *__restrict__ target,
                                                  const T *__restrict__ draft,
                                                  const float *__restrict__ temperature,
@@ -597,14 +605,24 @@ __global__ void SPECDEC_SWEEP_BOUNDS k_row_stats(const T *__restrict__ target,
     }
   }
   __syncthreads();
-  cudaGridDependencySynchronize();
+  const bool late = LATE && g.late_sync;
+  if (!late) cudaGridDependencySynchronize();
   // the dependent finish pass may be placed now; it reads this kernel's
   // results only after its own cudaGridDependencySynchronize
   cudaTriggerProgrammaticLaunchCompletion();
   // the arrival tickets of the finish pass start at 0
-  if (blockIdx.x == 0)
+  if (blockIdx.x == 0 && !late)
     for (int i = threadIdx.x; i < g.nb; i += blockDim.x) tickets[i] = 0u;
-  if (t0 >= t1) return;
+  auto late_end = [&]() {
+    if (late && blockIdx.x == 0 && threadIdx.x == 0) {
+      cudaGridDependencySynchronize();
+      for (int i = 0; i < g.nb; ++i) tickets[i] = 0u;
+    }
+  };
+  if (t0 >= t1) {
+    late_end();
+    return;
+  }
 
   // The CTA's tiles [t0, t1) are walked as row segments: the tiles of one row
   // that fall in the range.  Inside a segment the full tiles come first (no
@@ -792,6 +810,7 @@ __global__ void SPECDEC_SWEEP_BOUNDS k_row_stats(const T *__restrict__ target,
       }
     }
   }
+  late_end();
 }
 
 // ---------------------------------------------------------------------------
@@ -2027,8 +2046,8 @@ struct Plan {
   Sweep chain;           // chained second stage: the final layer's K+1 rows (the
                          // intermediate's statistics are kept from the first stage)
   int slots_max;         // partial slots per row in the workspace (the stride of every sweep)
-  size_t off_part, off_rpart, off_cnt, off_state, off_info, off_dlogw, off_s1tok, off_s1n,
-      off_rstat, total;
+  size_t off_part, off_part2, off_rpart, off_cnt, off_state, off_info, off_dlogw, off_s1tok,
+      off_s1n, off_rstat, total, total_chained;
 };
 
 int num_sms() {
@@ -2131,6 +2150,11 @@ bool make_plan(int B, int K, int V, specdec_dtype dtype, int sms, Plan &pl) {
   pl.off_rstat = off;
   off = align256(off + sizeof(Partial) * (size_t)B * (K + 1));
   pl.total = off > 0 ? off : 256;
+  // the chained verify's second sweep writes its partials apart (the first
+  // stage's finish pass may still read its own): a region after the others,
+  // in the chained verify's workspace only
+  pl.off_part2 = pl.total;
+  pl.total_chained = align256(pl.total + sizeof(Partial) * (size_t)pl.chain.rows * pl.slots_max * CW);
   return true;
 }
 
@@ -2216,6 +2240,9 @@ struct PassOpts {
   int dbg_pstride = -1;          // positions per sequence of p_x / q_x (default K)
   Partial *save_t = nullptr;      // keep the target rows' statistics here (see FinishWindow)
   const Partial *dstat = nullptr; // the draft rows' statistics from an earlier pass
+  Partial *part = nullptr;        // the sweep's partials (default: the workspace's first region)
+  bool late_capable = false;      // run the sweep's LATE instantiation (see k_row_stats)
+  bool late_sync = false;         // ... and let it stream before its wait
 };
 
 template <typename T, int NTH>
@@ -2252,7 +2279,7 @@ specdec_status launch_pass(const void *tg, const void *dr, const int32_t *tok, c
                            cudaStream_t st) {
   const T *t = static_cast<const T *>(tg);
   const T *d = static_cast<const T *>(dr);
-  Partial *part = reinterpret_cast<Partial *>(ws + pl.off_part);
+  Partial *part = o.part ? o.part : reinterpret_cast<Partial *>(ws + pl.off_part);
   ResPartial *rp = reinterpret_cast<ResPartial *>(ws + pl.off_rpart);
   unsigned *cnt = reinterpret_cast<unsigned *>(ws + pl.off_cnt);
   const int d_rows = o.d_rows > 0 ? o.d_rows : K;
@@ -2275,10 +2302,13 @@ specdec_status launch_pass(const void *tg, const void *dr, const int32_t *tok, c
   // per-CTA partials where many CTAs share a row (small batches): the finish
   // pass then reads fewer; otherwise one per warp and no CTA barrier
   g.pcw = sw.slots > kCtaCombineSlots ? 1 : CW;
+  g.late_sync = o.late_sync ? 1 : 0;
   cudaError_t e = cudaSuccess;
   {
     LaunchTimer lt(KID_STATS, st);
-    auto kern = pl.U == 4 ? k_row_stats<T, 4> : k_row_stats<T, 1>;
+    auto kern = o.late_capable
+                    ? (pl.U == 4 ? k_row_stats<T, 4, true> : k_row_stats<T, 1, true>)
+                    : (pl.U == 4 ? k_row_stats<T, 4> : k_row_stats<T, 1>);
     const size_t smem = (size_t)NSTAGE * NTC * pl.U * 16;
     // the sweep assumes its CTAs are co-resident only for speed, not for
     // progress: nothing waits on another CTA
@@ -2344,6 +2374,7 @@ specdec_status launch_chained(const void *fin, const void *inter, const void *dr
   Partial *rstat = reinterpret_cast<Partial *>(ws + pl.off_rstat);
   PassOpts o1;
   o1.save_t = rstat;  // the intermediate rows' statistics, for the second stage
+  o1.late_capable = true;
   specdec_status s = launch_pass<T>(inter, dr, tok, ua1, ur1, temp, B, K, V, pl, pl.full, o1, ws,
                                     nullptr, s1_tok, s1_n, st);
   if (s != SPECDEC_OK) return s;
@@ -2354,6 +2385,12 @@ specdec_status launch_chained(const void *fin, const void *inter, const void *dr
   o.emit_count = 1;
   o.dstat = rstat;  // the second stage sweeps the final layer's rows only
   o.dbg_pstride = K + 1;
+  // The final layer's logits are written by no kernel of this call: the
+  // second sweep streams them at once, while the first stage's finish pass
+  // still draws, into partials of its own.
+  o.part = reinterpret_cast<Partial *>(ws + pl.off_part2);
+  o.late_capable = true;
+  o.late_sync = true;
   return launch_pass<T>(fin, inter, s1_tok, ua2, ur2, temp, B, K, V, pl, pl.chain, o, ws,
                         dbg2, out_tokens, out_emitted, st);
 }
@@ -2652,7 +2689,7 @@ specdec_status specdec_verify_chained_ex(
   if (!make_plan(B, K, V, dtype, num_sms(), pl)) return SPECDEC_EINVAL;
   void *ws = nullptr;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  s = ensure_buf(g_ws, pl.total, st, &ws);
+  s = ensure_buf(g_ws, pl.total_chained, st, &ws);
   if (s != SPECDEC_OK) return s;
   char *w = static_cast<char *>(ws);
   int32_t *s1t = stage1_tokens ? stage1_tokens : reinterpret_cast<int32_t *>(w + pl.off_s1tok);
