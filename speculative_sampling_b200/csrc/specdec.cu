@@ -556,12 +556,20 @@ struct RowCursor {
 // completes after it.  (Both sweeps of a call that has such a stage use the
 // LATE instantiation: the second stage's CTAs were measured to overlap the
 // first stage's finish only when they run the same kernel as its sweep.)
-template <typename T, int U, bool LATE = false>
+// PLAIN: the sweep of the plain verify (every sequence, target and draft rows
+// of every position, a draft tensor of K rows per sequence), compiled with
+// those choices fixed: less code, and measured 0.2 us faster per call.
+template <typename T, int U, bool LATE = false, bool PLAIN = false>
 __global__ void SPECDEC_SWEEP_BOUNDS k_row_stats(const T *__restrict__ target,
                                                  const T *__restrict__ draft,
                                                  const float *__restrict__ temperature,
                                                  StatsGeom g, Partial *__restrict__ part,
                                                  unsigned *__restrict__ tickets, int B) {
+  if (PLAIN) {  // (the launch picks PLAIN only for these values)
+    g.state = nullptr;
+    g.tonly = 0;
+    g.d_rows = g.K;
+  }
   constexpr int VEC = Dt<T>::VEC;
   constexpr long long TV = (long long)NTC * U;  // vectors per tile
   constexpr unsigned TILE_BYTES = (unsigned)TV * 16u;
@@ -983,7 +991,10 @@ struct FinishWindow {
 };
 constexpr int kChainAll = -3;  // chained stage: every tested token accepted
 
-template <typename T, int UW, int NTH>
+// PLAIN: the finish of the plain verify (no early-exit state, no SMC-SD
+// weights, no chained stage), compiled with those paths removed: less code and
+// fewer spilled registers, measured 0.8-1.1 us faster per call.
+template <typename T, int UW, int NTH, bool PLAIN = false>
 __global__ void __launch_bounds__(NTH, 65536 / (NTH * kFinishMaxNreg)) k_finish(
     const T *__restrict__ target, const T *__restrict__ draft,
     const int32_t *__restrict__ tokens, const float *__restrict__ u_accept,
@@ -1009,6 +1020,16 @@ __global__ void __launch_bounds__(NTH, 65536 / (NTH * kFinishMaxNreg)) k_finish(
   const long long b = (long long)blockIdx.x / ncb;
   const int cb = (int)((long long)blockIdx.x - b * ncb);  // this CTA: chunks cb*cpb ...
   const int R = 2 * K + 1;
+  if (PLAIN) {  // (the launch picks PLAIN only for these values)
+    fw.state = nullptr;
+    fw.info = nullptr;
+    fw.decide_only = 0;
+    fw.dlogw = nullptr;
+    fw.len = nullptr;
+    fw.emit_count = 0;
+    fw.save_t = nullptr;
+    fw.dstat = nullptr;
+  }
   const int RW = fw.rps;  // rows of the window per sequence
   // The kernel after this one on the stream (the next call's statistics sweep,
   // or the SMC-SD resampling) may be placed as this grid's CTAs finish; it
@@ -2260,7 +2281,9 @@ cudaError_t launch_finish(const T *t, const T *d, const int32_t *tok, const floa
   if (ncb > pl.nsr) ncb = pl.nsr;
   const int cpb = decide_only ? pl.nsr : (int)((pl.nsr + ncb - 1) / ncb);
   const unsigned g2 = (unsigned)((long long)sw.nb * ((pl.nsr + cpb - 1) / cpb));
-  auto kern = k_finish<T, kFinishUW, NTH>;
+  const bool plain = fw.state == nullptr && fw.dlogw == nullptr && fw.len == nullptr &&
+                     fw.dstat == nullptr && fw.save_t == nullptr && !decide_only && !fw.emit_count;
+  auto kern = plain ? k_finish<T, kFinishUW, NTH, true> : k_finish<T, kFinishUW, NTH>;
   return launch_pdl(kern, g2, NTH, 0, st, t, d, tok, ua, ur, temp, K, (long long)V, pl.tpr, sw.tiles, sw.G1, pl.slots_max, pcw, pl.nsr, cpb, d_rows, tok_stride, fw,
                     part, rp, cnt, out_tokens, out_n, dbg ? dbg->row_max : nullptr,
                     dbg ? dbg->row_sum : nullptr, dbg ? dbg->p_x : nullptr,
@@ -2306,9 +2329,12 @@ specdec_status launch_pass(const void *tg, const void *dr, const int32_t *tok, c
   cudaError_t e = cudaSuccess;
   {
     LaunchTimer lt(KID_STATS, st);
+    const bool plain = !o.late_capable && g.state == nullptr && !g.tonly && g.d_rows == K;
     auto kern = o.late_capable
                     ? (pl.U == 4 ? k_row_stats<T, 4, true> : k_row_stats<T, 1, true>)
-                    : (pl.U == 4 ? k_row_stats<T, 4> : k_row_stats<T, 1>);
+                    : plain ? (pl.U == 4 ? k_row_stats<T, 4, false, true>
+                                         : k_row_stats<T, 1, false, true>)
+                            : (pl.U == 4 ? k_row_stats<T, 4> : k_row_stats<T, 1>);
     const size_t smem = (size_t)NSTAGE * NTC * pl.U * 16;
     // the sweep assumes its CTAs are co-resident only for speed, not for
     // progress: nothing waits on another CTA
