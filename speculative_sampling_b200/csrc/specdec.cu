@@ -2135,7 +2135,17 @@ bool make_plan(int B, int K, int V, specdec_dtype dtype, int sms, Plan &pl) {
   }
   if (tpr < 1) tpr = 1;
   pl.tpr = (int)tpr;
-  pl.full = make_sweep(B, 0, K, 1, pl.tpr, cap);
+  // Small batches (4 KB tiles): a grid of m CTAs per row, so that every CTA's
+  // range lies inside one row (one partial, no row changes), with at least 3
+  // tiles per CTA and at most kStatsCtasPerSm CTAs per SM.  Measured against
+  // the full 444-CTA grid: B = 1 15.9 -> 13.9 us, B = 4 17.9 -> 16.3 us.
+  long long cap_full = cap;
+  if (pl.U == 1) {
+    long long m = cap / rows;
+    if (m > tpr / 3) m = tpr / 3;
+    if (m >= 1) cap_full = rows * m;
+  }
+  pl.full = make_sweep(B, 0, K, 1, pl.tpr, cap_full);
   const int P = early_split(K);
   pl.first = make_sweep(B, 0, P, 0, pl.tpr, cap);
   pl.second = make_sweep(B, P, K - P, 1, pl.tpr, cap);
