@@ -2078,10 +2078,19 @@ int num_sms() {
 }
 
 // partition of a sweep's tiles over its CTAs and the partial slots per row:
-// the most CTAs whose tile ranges meet one row
-void sweep_partition(Sweep &w, int tpr, long long cap) {
+// the most CTAs whose tile ranges meet one row.  With small (4 KB) tiles the
+// grid is m CTAs per row, so that every CTA's range lies inside one row (one
+// partial, no row changes), with at least 3 tiles per CTA and at most `cap`
+// CTAs.  Measured against the full 444-CTA grid: B = 1 15.9 -> 13.9 us per
+// call, B = 4 17.9 -> 16.3 us.
+void sweep_partition(Sweep &w, int tpr, long long cap, bool small_tiles) {
   w.rows = (long long)w.nb * w.rps;
   w.tiles = w.rows * tpr;
+  if (small_tiles && w.rows > 0) {
+    long long m = cap / w.rows;
+    if (m > tpr / 3) m = tpr / 3;
+    if (m >= 1) cap = w.rows * m;
+  }
   w.G1 = w.tiles < cap ? w.tiles : cap;
   if (w.G1 < 1) w.G1 = 1;
   const long long minr = w.tiles / w.G1;  // shortest range
@@ -2090,7 +2099,7 @@ void sweep_partition(Sweep &w, int tpr, long long cap) {
 
 // A sweep over nb sequences: the target and draft rows of positions
 // p0 .. p0+np-1 and, with `bonus`, the target's row K.
-Sweep make_sweep(int nb, int p0, int np, int bonus, int tpr, long long cap) {
+Sweep make_sweep(int nb, int p0, int np, int bonus, int tpr, long long cap, bool small_tiles) {
   Sweep w;
   w.p0 = p0;
   w.np = np;
@@ -2098,16 +2107,16 @@ Sweep make_sweep(int nb, int p0, int np, int bonus, int tpr, long long cap) {
   w.rps = 2 * np + bonus;
   w.tonly = 0;
   w.nb = nb;
-  sweep_partition(w, tpr, cap);
+  sweep_partition(w, tpr, cap, small_tiles);
   return w;
 }
 
 // A sweep over the target tensor's rows p0 .. p0+np-1 only.
-Sweep make_target_sweep(int nb, int p0, int np, int tpr, long long cap) {
-  Sweep w = make_sweep(nb, p0, np, 0, tpr, cap);
+Sweep make_target_sweep(int nb, int p0, int np, int tpr, long long cap, bool small_tiles) {
+  Sweep w = make_sweep(nb, p0, np, 0, tpr, cap, small_tiles);
   w.tonly = 1;
   w.rps = np;
-  sweep_partition(w, tpr, cap);
+  sweep_partition(w, tpr, cap, small_tiles);
   return w;
 }
 
@@ -2135,21 +2144,12 @@ bool make_plan(int B, int K, int V, specdec_dtype dtype, int sms, Plan &pl) {
   }
   if (tpr < 1) tpr = 1;
   pl.tpr = (int)tpr;
-  // Small batches (4 KB tiles): a grid of m CTAs per row, so that every CTA's
-  // range lies inside one row (one partial, no row changes), with at least 3
-  // tiles per CTA and at most kStatsCtasPerSm CTAs per SM.  Measured against
-  // the full 444-CTA grid: B = 1 15.9 -> 13.9 us, B = 4 17.9 -> 16.3 us.
-  long long cap_full = cap;
-  if (pl.U == 1) {
-    long long m = cap / rows;
-    if (m > tpr / 3) m = tpr / 3;
-    if (m >= 1) cap_full = rows * m;
-  }
-  pl.full = make_sweep(B, 0, K, 1, pl.tpr, cap_full);
+  const bool small = pl.U == 1;
+  pl.full = make_sweep(B, 0, K, 1, pl.tpr, cap, small);
   const int P = early_split(K);
-  pl.first = make_sweep(B, 0, P, 0, pl.tpr, cap);
-  pl.second = make_sweep(B, P, K - P, 1, pl.tpr, cap);
-  pl.chain = make_target_sweep(B, 0, K + 1, pl.tpr, cap);
+  pl.first = make_sweep(B, 0, P, 0, pl.tpr, cap, small);
+  pl.second = make_sweep(B, P, K - P, 1, pl.tpr, cap, small);
+  pl.chain = make_target_sweep(B, 0, K + 1, pl.tpr, cap, small);
   pl.slots_max = pl.full.slots;
   for (const Sweep *w : {&pl.first, &pl.second, &pl.chain})
     if (w->slots > pl.slots_max) pl.slots_max = w->slots;
