@@ -39,3 +39,17 @@ def test_reference_arm_prints_one_json_line():
 
 def test_reference_arm_other_ranks_exit_without_output():
     assert _run({"RANK": "1", "WORLD_SIZE": "2"}) == []
+
+
+def test_cuda_arm_fails_loudly_without_a_gpu():
+    """No silent fallback: without a CUDA device the product arm exits non-zero and
+    prints no result line."""
+    import pytest
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--steps", "1",
+                        "--warmup", "3", "--no-cpu-baseline"],
+                       capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode != 0
+    assert not any(l.startswith("{") for l in r.stdout.splitlines())
