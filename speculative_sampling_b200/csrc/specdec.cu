@@ -7,12 +7,14 @@
 // from Leviathan et al.").  This file is the B200 implementation:
 //
 //   k_row_stats     one pass over every logit row (B*(2K+1) rows of V): a
-//                   producer thread streams 16 KB tiles with TMA bulk copies
-//                   into a 3-stage shared-memory ring (full/empty mbarriers,
-//                   every wait bounded); 8 consumer warps fold them into
-//                   split-V softmax statistics (row max m, sum of 2^((z-m)*c))
-//                   and each CTA writes one partial per row segment.  It
-//                   streams the whole input once and is the HBM-bound kernel.
+//                   producer thread streams 16 KB tiles (4 KB for batches of
+//                   a few sequences) with TMA bulk copies into a 3-stage
+//                   shared-memory ring (full/empty mbarriers, every wait
+//                   bounded); 8 consumer warps fold them into split-V softmax
+//                   statistics (row max m, sum of 2^((z-m)*c)) and write, per
+//                   row segment, one partial per warp (or one per CTA where
+//                   many CTAs share a row).  It streams the whole input once
+//                   and is the HBM-bound kernel.
 //   k_finish        per sequence, on several CTAs: combines the partials of the
 //                   2K+1 rows in fp64, gathers p_i(x_i), q_i(x_i), tests
 //                   u*q < p on K lanes (__ballot_sync/__ffs), writes the
@@ -27,7 +29,9 @@
 // dependents early and waits for its predecessor
 // (cudaGridDependencySynchronize) only where it first needs its results; the
 // call's first kernel waits before it reads anything (the statistics sweep
-// only requests its first tiles into L2 before that).
+// only requests its first tiles into L2 before that; the chained verify's
+// second sweep, which reads only inputs no kernel of the call writes, streams
+// at once and waits at its end).
 //
 // Arithmetic: logits are widened exactly to fp32.  Exponentials are
 // 2^((z - m) * c) with c = log2(e)/T carried as an fp32 pair (hi + lo, with
@@ -187,8 +191,10 @@ __device__ __forceinline__ float half_max_nan(float v) {
 // ---------------------------------------------------------------------------
 // A sweep reads the rows of its window (every row of the batch, or some
 // positions of it), in sequence order, cut into tiles of CW*32*U 16-byte
-// vectors (16 KB for U = 4);
-// CTA g of a grid of G owns the contiguous tile range [g*T/G, (g+1)*T/G).
+// vectors (16 KB for U = 4, 4 KB for U = 1);
+// CTA g of a grid of G owns the contiguous tile range [g*T/G, (g+1)*T/G)
+// (with 4 KB tiles G is, where rows have 3 tiles or more, a multiple of the
+// rows, so each range lies in one row: see sweep_partition).
 //
 // Warp specialisation: one producer warp streams tiles with cp.async.bulk
 // (the TMA bulk-copy engine; each CTA copies only into its own shared memory)
@@ -2134,7 +2140,7 @@ bool make_plan(int B, int K, int V, specdec_dtype dtype, int sms, Plan &pl) {
   const long long rows = (long long)B * (2 * K + 1);
   const long long nvec_max = ((long long)V + pl.vec - 1) / pl.vec;
   // tiles of 4 vectors per consumer thread (16 KB); 1 vector per thread when
-  // 16 KB tiles would leave SMs idle (single-sequence batches)
+  // 16 KB tiles would leave SMs idle (batches of a few sequences)
   const long long cap = (long long)kStatsCtasPerSm * sms;
   long long tpr = (nvec_max + NTC * 4 - 1) / (NTC * 4);
   pl.U = 4;
