@@ -262,8 +262,10 @@ specdec_status specdec_topk_exclude(const void *logits, long long row_stride,
  * tensors, a draft token or the temperature, as in specdec_verify).
  * stage1_tokens [B, K+1] / stage1_num_accepted [B] (nullable) receive stage 1's
  * outputs.  K <= 31.  Device memory, asynchronous on `stream`, library-owned
- * workspace.  Two statistics sweeps: both tensors of stage 1, then the final
- * and intermediate tensors again for stage 2. */
+ * workspace.  Two statistics sweeps: the intermediate and draft tensors for
+ * stage 1, then the final layer's rows only for stage 2 (the intermediate
+ * rows' statistics are kept from stage 1); the second sweep starts streaming
+ * while stage 1's finish pass draws. */
 specdec_status specdec_verify_chained(
     const void *final_logits, const void *intermediate_logits, const void *draft_logits,
     const int32_t *draft_tokens, const float *u_accept1, const float *u_resample1,
