@@ -43,7 +43,9 @@
  * launch: a call's first kernel may be placed on the GPU while the kernel
  * before it on the stream is still running, but it reads no input and writes
  * nothing until that kernel has completed, so stream order holds for the
- * caller's producers of the inputs.  The call's last kernel lets a following
+ * caller's producers of the inputs.  (Before that wait the statistics sweep
+ * may ask for its first input tiles to be brought into L2: a cache hint that
+ * reads nothing, and L2 stays coherent with whatever that kernel writes.)  The call's last kernel lets a following
  * kernel launched with programmatic serialisation start early; such a kernel
  * must call cudaGridDependencySynchronize() before it reads the outputs (as
  * the programming model requires of it anyway).  The logit pointers must be
